@@ -1,0 +1,577 @@
+// Attention on tcgen05 tensor cores: the dense warm-up pass with per-query
+// entropy, and exact block-sparse attention over a CSR block list.
+//
+// Token Radius Attention summary (gist.science 2608.02504): §2 "TRA pipeline"
+// step 1 (entropy of every query from a dense warm-up pass), §3 contribution 3
+// (fused entropy kernel), efficient execution (block-sparse attention over the
+// kept query-block x key-block pairs, reused across sparse steps).
+//
+// One CTA computes 128 query rows of one head against a list of key blocks
+// (all blocks for the dense pass; the CSR row for the sparse pass; when
+// query blocks are smaller than 128 rows, the union of the rows' lists with
+// per-row masking).  Warp roles:
+//   warp 0      TMA producer: Q once, then K and V tiles into a 2-stage ring
+//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
+//               score buffers, O += P_j V_j into a TMEM accumulator
+//   warp 2      allocates / frees tensor memory
+//   warps 4..7  softmax: thread i owns query row i (TMEM lane i); reads S_j,
+//               keeps the running max m, Z = sum 2^(u-m) and
+//               A = sum 2^(u-m) (u-m) (u = s*log2 e), writes P_j (bf16) to
+//               shared memory in the MMA's swizzled layout, rescales O when
+//               the max grows by more than 2^8, and writes O / Z, the entropy
+//               H = ln Z - ln 2 * A / Z and LSE = ln 2 * (m + log2 Z).
+// S_{j+1} runs on the tensor cores while the softmax of block j runs.
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <mutex>
+
+#include "ptx.cuh"
+#include "tra_internal.h"
+
+namespace tra {
+namespace {
+
+constexpr int BM = 128;                    // query rows per CTA
+constexpr int kThreads = 256;              // 8 warps
+constexpr int kMaxUnion = 1024;            // key blocks of a merged list
+constexpr int kMaxGroups = 8;              // query blocks per CTA (128 / 16)
+constexpr float kRescaleLog2 = 8.0f;       // lazy rescale threshold (log2 units)
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kLog2e = 1.44269504088896340736f;
+
+__host__ __device__ constexpr int pow2_at_least(int x) {
+  int p = 32;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+template <int D, int BK>
+struct Cfg {
+  static constexpr int NS = 2;                          // K and V ring depth
+  static constexpr int KCH = D / 64;                    // 128-byte groups of a Q/K/V row
+  static constexpr int PCH = (BK + 63) / 64;            // 128-byte groups of a P row
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BK * D * 2;
+  static constexpr int P_BYTES = PCH * BM * 128;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + NS * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int NUM_BARS = 1 + 4 * NS + 6;
+  static constexpr int OFF_MISC = OFF_BAR + 256;
+  static constexpr int OFF_LIST = OFF_MISC + 64;
+  static constexpr int OFF_QBMAP = OFF_LIST + kMaxUnion * 4;
+  static constexpr int USED = OFF_QBMAP + kMaxGroups * 32 * 4;
+  static constexpr int TMEM_COLS = pow2_at_least(2 * BK + D);
+  // 512 tensor-memory columns fill an SM: make sure a second CTA cannot be
+  // co-resident (it would only wait for the first to free the columns).
+  static constexpr int SMEM = (TMEM_COLS == 512 && USED < 120 * 1024 ? 120 * 1024 : USED) + 1024;
+  static_assert(Q_BYTES % 1024 == 0 && KV_BYTES % 1024 == 0, "swizzle atoms need 1 KiB alignment");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(NUM_BARS * 8 <= 256, "barrier area");
+};
+
+struct Params {
+  int N, nqb, nkb, bq, G;
+  float scale_log2;
+  const int* row_ptr;
+  const int* col_idx;
+  __nv_bfloat16* O;
+  float* H;
+  float* lse;
+  int* err;
+};
+
+__device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
+        "=f"(v[7]), "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]),
+        "=f"(v[14]), "=f"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16f(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
+      "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]),
+      "f"(v[15])
+      : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void freg_fence(float* v) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// Bounded wait that ignores the abort flag (used to drain copies in flight).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > 500000000ull) break;
+  }
+}
+
+template <int D, int BK, bool DENSE>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using C = Cfg<D, BK>;
+  constexpr int NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::OFF_Q;
+  const uint32_t sK = sbase + C::OFF_K;
+  const uint32_t sV = sbase + C::OFF_V;
+  const uint32_t sP = sbase + C::OFF_P;
+  const uint32_t bars = sbase + C::OFF_BAR;
+  const uint32_t bar_q = bars;
+  auto k_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto k_empty = [&](int s) { return bars + 8u * (1 + NS + s); };
+  auto v_full = [&](int s) { return bars + 8u * (1 + 2 * NS + s); };
+  auto v_empty = [&](int s) { return bars + 8u * (1 + 3 * NS + s); };
+  auto s_full = [&](int b) { return bars + 8u * (1 + 4 * NS + b); };
+  auto s_free = [&](int b) { return bars + 8u * (3 + 4 * NS + b); };
+  const uint32_t p_full = bars + 8u * (5 + 4 * NS);
+  const uint32_t pv_done = bars + 8u * (6 + 4 * NS);
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
+  // misc[0] tmem base, misc[1] abort, misc[2] block count, misc[3] CSR start
+  volatile int* abort = misc + 1;
+  int* list = reinterpret_cast<int*>(smem + C::OFF_LIST);
+  uint32_t* qbmap = reinterpret_cast<uint32_t*>(smem + C::OFF_QBMAP);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int qt = blockIdx.x, h = blockIdx.y;
+
+  if (tid == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full(b), 1);
+      mbar_init(s_free(b), 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    fence_barrier_init();
+    misc[1] = 0;
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(const_cast<int*>(misc)), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    tma_prefetch_map(&tmQ);
+    tma_prefetch_map(&tmK);
+    tma_prefetch_map(&tmV);
+  }
+
+  // ---- key-block list of this CTA
+  if constexpr (DENSE) {
+    if (tid == 0) misc[2] = p.nkb;
+  } else {
+    const int* rp = p.row_ptr + static_cast<size_t>(h) * (p.nqb + 1);
+    if (p.G == 1) {
+      if (tid == 0) {
+        const int st = rp[qt], en = rp[qt + 1];
+        int n = en - st;
+        if (st < 0 || n < 0 || n > p.nkb) {
+          n = 0;
+          atomicCAS(p.err, 0, kErrBadCsr);
+        }
+        misc[2] = n;
+        misc[3] = st;
+      }
+    } else {
+      const int nkbw = (p.nkb + 31) >> 5;
+      for (int i = tid; i < kMaxGroups * 32; i += kThreads) qbmap[i] = 0u;
+      __syncthreads();
+      for (int g = 0; g < p.G; ++g) {
+        const int qb = qt * p.G + g;
+        if (qb >= p.nqb) break;
+        const int st = rp[qb], en = rp[qb + 1];
+        if (st < 0 || en - st < 0 || en - st > p.nkb) {
+          if (tid == 0) atomicCAS(p.err, 0, kErrBadCsr);
+          continue;
+        }
+        for (int e = st + tid; e < en; e += kThreads) {
+          const int kb = p.col_idx[e];
+          if (kb >= 0 && kb < p.nkb) atomicOr(&qbmap[g * 32 + (kb >> 5)], 1u << (kb & 31));
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {
+        int run = 0;
+        for (int base = 0; base < nkbw; base += 32) {
+          const int w = base + lane;
+          uint32_t word = 0;
+          if (w < nkbw)
+            for (int g = 0; g < p.G; ++g) word |= qbmap[g * 32 + w];
+          const int c = __popc(word);
+          int incl = c;
+          for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+          }
+          int pos = run + incl - c;
+          while (word) {
+            const int b = __ffs(word) - 1;
+            word &= word - 1;
+            list[pos++] = w * 32 + b;
+          }
+          run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) misc[2] = run;
+      }
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+  const int nblk = misc[2];
+  const int csr_start = misc[3];
+
+  auto kb_at = [&](int j) -> int {
+    if constexpr (DENSE) {
+      return j;
+    } else {
+      return p.G == 1 ? __ldg(p.col_idx + csr_start + j) : list[j];
+    }
+  };
+
+  if (warp == 0) {
+    // ===================================================== TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * (BM * 128), &tmQ, c * 64, qt * BM, h, bar_q);
+      int issued = 0;
+      for (int j = 0; j < nblk; ++j) {
+        const int s = j % NS;
+        const uint32_t ph = (j / NS) & 1;
+        const int kb = kb_at(j);
+        if (!mbar_wait(k_empty(s), ph ^ 1u, abort, p.err, kErrWaitKEmpty)) break;
+        mbar_arrive_expect_tx(k_full(s), C::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sK + s * C::KV_BYTES + c * (BK * 128), &tmK, c * 64, kb * BK, h, k_full(s));
+        if (!mbar_wait(v_empty(s), ph ^ 1u, abort, p.err, kErrWaitVEmpty)) {
+          issued = -(j + 1);  // K of block j in flight, V not
+          break;
+        }
+        mbar_arrive_expect_tx(v_full(s), C::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sV + s * C::KV_BYTES + c * (BK * 128), &tmV, c * 64, kb * BK, h, v_full(s));
+        issued = j + 1;
+      }
+      if (*abort) {
+        // let every copy still in flight land before the CTA can exit
+        drain_wait(bar_q, 0);
+        const int kdone = issued >= 0 ? issued : -issued;
+        const int vdone = issued >= 0 ? issued : -issued - 1;
+        for (int j = (kdone > NS ? kdone - NS : 0); j < kdone; ++j)
+          drain_wait(k_full(j % NS), (j / NS) & 1);
+        for (int j = (vdone > NS ? vdone - NS : 0); j < vdone; ++j)
+          drain_wait(v_full(j % NS), (j / NS) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ===================================================== MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BK, 0, 0);
+      constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, D, 0, 1);
+      const uint32_t tO = tmem + 2 * BK;
+      auto issue_pv = [&](int i) -> bool {
+        const int s = i % NS;
+        if (!mbar_wait(p_full, i & 1, abort, p.err, kErrWaitPFull)) return false;
+        if (!mbar_wait(v_full(s), (i / NS) & 1, abort, p.err, kErrWaitVFull)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          const uint64_t a = smem_desc_sw128(sP + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024);
+          const uint64_t b = smem_desc_sw128(sV + s * C::KV_BYTES + k * 16 * 128, BK * 128, 1024);
+          mma_bf16_ss(tO, a, b, kIdescPV, (i > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(v_empty(s));
+        mma_commit(pv_done);
+        return true;
+      };
+      bool ok = mbar_wait(bar_q, 0, abort, p.err, kErrWaitQ);
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int s = j % NS;
+        const int b = j & 1;
+        if (!mbar_wait(k_full(s), (j / NS) & 1, abort, p.err, kErrWaitKFull)) { ok = false; break; }
+        if (!mbar_wait(s_free(b), ((j >> 1) & 1) ^ 1u, abort, p.err, kErrWaitSFree)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tS = tmem + b * BK;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t a = smem_desc_sw128(sQ + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              smem_desc_sw128(sK + s * C::KV_BYTES + (k >> 2) * (BK * 128) + (k & 3) * 32, 16, 1024);
+          mma_bf16_ss(tS, a, bd, kIdescQK, k > 0 ? 1u : 0u);
+        }
+        mma_commit(k_empty(s));
+        mma_commit(s_full(b));
+        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok && nblk > 0) ok = issue_pv(nblk - 1);
+      if (!ok) {
+        // wait for every MMA issued so far before tensor memory is freed
+        const uint32_t drain = bars + 8u * (C::NUM_BARS);
+        mbar_init(drain, 1);
+        fence_barrier_init();
+        mma_commit(drain);
+        drain_wait(drain, 0);
+      }
+    }
+  } else if (warp >= 4) {
+    // ===================================================== softmax / epilogue
+    const int row = tid - 128;
+    const uint32_t tl = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int qpos = qt * BM + row;
+    const bool valid_row = qpos < p.N;
+    const int g = DENSE ? 0 : row / p.bq;
+    float m_ref = -INFINITY, Z = 0.f, A = 0.f;
+    bool ok = true;
+    float sv[BK];
+    for (int j = 0; j < nblk; ++j) {
+      const int b = j & 1;
+      const int kb = kb_at(j);
+      ok = mbar_wait(s_full(b), (j >> 1) & 1, abort, p.err, kErrWaitSFull);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < BK / 16; ++c) tmem_ld16f(tmem + tl + b * BK + c * 16, sv + c * 16);
+      tmem_wait_ld();
+      freg_fence<BK>(sv);
+      tc_fence_before();
+      mbar_arrive(s_free(b));
+
+      int nvalid = p.N - kb * BK;
+      if constexpr (!DENSE) {
+        if (kb < 0 || kb >= p.nkb) nvalid = 0;
+        else if (p.G > 1 && !((qbmap[g * 32 + (kb >> 5)] >> (kb & 31)) & 1u)) nvalid = 0;
+      }
+      float bmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BK; ++c) {
+        const float u = c < nvalid ? sv[c] * p.scale_log2 : -INFINITY;
+        sv[c] = u;
+        bmax = fmaxf(bmax, u);
+      }
+      const float m_new = fmaxf(m_ref, bmax);
+      float alpha = 1.f;
+      bool o_rescale = false;
+      if (m_new > m_ref + kRescaleLog2) {
+        if (m_ref != -INFINITY) {
+          alpha = exp2f(m_ref - m_new);
+          A = alpha * (A + (m_ref - m_new) * Z);
+          Z *= alpha;
+          o_rescale = j > 0;
+        }
+        m_ref = m_new;
+      }
+      const float mc = (m_ref == -INFINITY) ? 0.f : m_ref;
+      float zs = 0.f, as = 0.f;
+#pragma unroll
+      for (int c = 0; c < BK; ++c) {
+        const float x = sv[c] - mc;
+        const float pr = exp2f(x);
+        zs += pr;
+        if constexpr (DENSE) as += pr > 0.f ? pr * x : 0.f;
+        sv[c] = pr;
+      }
+      Z += zs;
+      A += as;
+
+      if (j > 0) {
+        ok = mbar_wait(pv_done, (j - 1) & 1, abort, p.err, kErrWaitPVDone);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, o_rescale)) {
+        const float a = o_rescale ? alpha : 1.f;
+#pragma unroll
+        for (int c = 0; c < D; c += 16) {
+          float o[16];
+          tmem_ld16f(tmem + tl + 2 * BK + c, o);
+          tmem_wait_ld();
+          freg_fence<16>(o);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] *= a;
+          tmem_st16f(tmem + tl + 2 * BK + c, o);
+        }
+        tmem_wait_st();
+      }
+#pragma unroll
+      for (int c8 = 0; c8 < BK / 8; ++c8) {
+        const uint32_t addr = sP + (c8 >> 3) * (BM * 128) + row * 128 + (((c8 & 7) ^ (row & 7)) << 4);
+        st_shared_v4(addr, pack_bf16(sv[c8 * 8 + 0], sv[c8 * 8 + 1]),
+                     pack_bf16(sv[c8 * 8 + 2], sv[c8 * 8 + 3]),
+                     pack_bf16(sv[c8 * 8 + 4], sv[c8 * 8 + 5]),
+                     pack_bf16(sv[c8 * 8 + 6], sv[c8 * 8 + 7]));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok && nblk > 0) {
+      ok = mbar_wait(pv_done, (nblk - 1) & 1, abort, p.err, kErrWaitPVDone);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    tc_fence_after();
+    const float inv = Z > 0.f ? 1.f / Z : 0.f;
+    __nv_bfloat16* orow = p.O + (static_cast<size_t>(h) * p.N + (valid_row ? qpos : 0)) * D;
+    if (ok && nblk > 0) {
+#pragma unroll
+      for (int c = 0; c < D; c += 16) {
+        float o[16];
+        tmem_ld16f(tmem + tl + 2 * BK + c, o);
+        tmem_wait_ld();
+        freg_fence<16>(o);
+        if (valid_row) {
+          uint4 w0, w1;
+          w0.x = pack_bf16(o[0] * inv, o[1] * inv);
+          w0.y = pack_bf16(o[2] * inv, o[3] * inv);
+          w0.z = pack_bf16(o[4] * inv, o[5] * inv);
+          w0.w = pack_bf16(o[6] * inv, o[7] * inv);
+          w1.x = pack_bf16(o[8] * inv, o[9] * inv);
+          w1.y = pack_bf16(o[10] * inv, o[11] * inv);
+          w1.z = pack_bf16(o[12] * inv, o[13] * inv);
+          w1.w = pack_bf16(o[14] * inv, o[15] * inv);
+          reinterpret_cast<uint4*>(orow + c)[0] = w0;
+          reinterpret_cast<uint4*>(orow + c)[1] = w1;
+        }
+      }
+    } else if (valid_row) {
+      for (int c = 0; c < D; c += 8) reinterpret_cast<uint4*>(orow + c)[0] = make_uint4(0, 0, 0, 0);
+    }
+    if (valid_row) {
+      const size_t idx = static_cast<size_t>(h) * p.N + qpos;
+      if (DENSE && p.H != nullptr) p.H[idx] = Z > 0.f ? logf(Z) - kLn2 * (A / Z) : NAN;
+      if (p.lse != nullptr) p.lse[idx] = Z > 0.f ? kLn2 * (m_ref + log2f(Z)) : -INFINITY;
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// [heads, N, d] bf16 as a 3D tensor (d, N, heads); boxes of 64 x rows x 1,
+// 128-byte swizzle; rows past N read as zeros.
+bool make_map(CUtensorMap* map, const void* base, int d, int N, int heads, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * d * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int BK, bool DENSE>
+cudaError_t launch_cfg(const AttnArgs& a, const Params& prm, cudaStream_t stream) {
+  using C = Cfg<D, BK>;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.Q, D, a.N, a.heads, BM) || !make_map(&mk, a.K, D, a.N, a.heads, BK) ||
+      !make_map(&mv, a.V, D, a.N, a.heads, BK))
+    return cudaErrorInvalidValue;
+  auto kern = attn_kernel<D, BK, DENSE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((a.N + BM - 1) / BM, a.heads);
+  kern<<<grid, kThreads, C::SMEM, stream>>>(mq, mk, mv, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
+  Params prm;
+  prm.N = a.N;
+  const int bk = a.dense ? 128 : a.block_k;
+  const int bq = a.dense ? 128 : a.block_q;
+  prm.nqb = (a.N + bq - 1) / bq;
+  prm.nkb = (a.N + bk - 1) / bk;
+  prm.bq = bq;
+  prm.G = BM / bq;
+  prm.scale_log2 = a.scale * kLog2e;
+  prm.row_ptr = a.row_ptr;
+  prm.col_idx = a.col_idx;
+  prm.O = static_cast<__nv_bfloat16*>(a.O);
+  prm.H = a.H;
+  prm.lse = a.lse;
+  prm.err = device_error_word();
+  if (a.dense) {
+    if (a.d == 128) return launch_cfg<128, 128, true>(a, prm, stream);
+    return launch_cfg<64, 128, true>(a, prm, stream);
+  }
+  if (a.d == 128) {
+    if (bk == 128) return launch_cfg<128, 128, false>(a, prm, stream);
+    if (bk == 64) return launch_cfg<128, 64, false>(a, prm, stream);
+    return launch_cfg<128, 16, false>(a, prm, stream);
+  }
+  if (bk == 128) return launch_cfg<64, 128, false>(a, prm, stream);
+  if (bk == 64) return launch_cfg<64, 64, false>(a, prm, stream);
+  return launch_cfg<64, 16, false>(a, prm, stream);
+}
+
+}  // namespace tra

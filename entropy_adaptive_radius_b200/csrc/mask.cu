@@ -1,0 +1,411 @@
+// Fused radius mask -> block-sparse CSR (Token Radius Attention summary, §2
+// "TRA pipeline", efficient execution: distance computation, radius compare,
+// block pruning and token voting fused into one kernel that emits a regular
+// query-block x key-block mask).
+//
+// Token mask: key j is in query i's support when dx^2 + dy^2 <= R2 with
+// R2 = fl32(fl32(r_i * phi[|t_j - t_i|])^2); non-finite radii keep every key.
+// Distances are integers, so the compare is done exactly as
+// dx^2 + dy^2 <= floor(R2) (R2 clamped to 2^30, above any grid distance).
+//
+// Four launches:
+//  1. footprint: for every key block, the rows (t, y, [x_lo, x_hi]) its tokens
+//     cover and per-frame bounding boxes.  A contiguous run of tile-major
+//     positions covers, for each (t, y), one contiguous x interval; the kernel
+//     verifies this per block and otherwise marks the block for token-by-token
+//     testing.
+//  2. votes: one CTA per (head, query block).  Each CTA bounds, for every key
+//     frame, the union of its queries' disks by a box; a key block whose
+//     per-frame boxes miss those boxes has no votes and is pruned (lanes over
+//     key blocks).  Survivors are counted exactly (lanes over queries): for a
+//     query and a key row the number of keys inside the disk is the overlap of
+//     [x_lo, x_hi] with [x_q - s, x_q + s], s = isqrt(floor(R2) - dy^2); with a
+//     vote threshold of 1 an existence test replaces the count.  Counting stops
+//     once the threshold is reached (only "votes >= threshold" is needed).
+//  3. scan: exclusive prefix sum of the per-row kept counts -> row_ptr, nnz.
+//  4. compact: kept bits -> ascending col_idx.
+#include "tra_internal.h"
+
+namespace tra {
+namespace {
+
+constexpr int kMaxSeg = 4;  // per-frame boxes kept per key block (more: no pruning)
+constexpr int kVoteThreads = 128;
+constexpr int kRsqCap = 1 << 30;
+
+struct MaskWs {
+  uint2* rows;      // [nkb * Bk]: x = t << 16 | y, y = x_lo << 16 | x_hi
+  int4* info;       // [nkb]: x = rows (-1: not row-contiguous), y = segments (-1: too many), z = tokens
+  int4* segs;       // [nkb * kMaxSeg]: x = t, y = y_lo << 16 | y_hi, z = x_lo << 16 | x_hi
+  uint32_t* bits;   // [heads * nqb * nkbw]
+  int* counts;      // [heads * nqb]
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct MaskDims {
+  int N, nqb, nkb, nkbw;
+};
+
+__host__ __device__ inline MaskDims mask_dims(const TileLayout& L, int bq, int bk) {
+  MaskDims m;
+  m.N = L.F * L.H * L.W;
+  m.nqb = (m.N + bq - 1) / bq;
+  m.nkb = (m.N + bk - 1) / bk;
+  m.nkbw = (m.nkb + 31) / 32;
+  return m;
+}
+
+size_t carve(const TileLayout& L, int heads, int bq, int bk, char* base, MaskWs* ws) {
+  const MaskDims m = mask_dims(L, bq, bk);
+  size_t off = 0;
+  const size_t rows = align256(sizeof(uint2) * static_cast<size_t>(m.nkb) * bk);
+  const size_t info = align256(sizeof(int4) * static_cast<size_t>(m.nkb));
+  const size_t segs = align256(sizeof(int4) * static_cast<size_t>(m.nkb) * kMaxSeg);
+  const size_t bits = align256(sizeof(uint32_t) * static_cast<size_t>(heads) * m.nqb * m.nkbw);
+  const size_t counts = align256(sizeof(int) * static_cast<size_t>(heads) * m.nqb);
+  if (ws) {
+    ws->rows = reinterpret_cast<uint2*>(base + off);
+    ws->info = reinterpret_cast<int4*>(base + off + rows);
+    ws->segs = reinterpret_cast<int4*>(base + off + rows + info);
+    ws->bits = reinterpret_cast<uint32_t*>(base + off + rows + info + segs);
+    ws->counts = reinterpret_cast<int*>(base + off + rows + info + segs + bits);
+  }
+  return rows + info + segs + bits + counts;
+}
+
+__device__ __forceinline__ int isqrt_floor(int m) {
+  int s = static_cast<int>(sqrtf(static_cast<float>(m)));
+  while (s * s > m) --s;
+  while ((s + 1) * (s + 1) <= m) ++s;
+  return s;
+}
+
+// floor(fl32(fl32(r * phi)^2)), clamped to 2^30 (also for +inf and NaN).
+__device__ __forceinline__ int radius_sq(float r, float phi) {
+  const float R = __fmul_rn(r, phi);
+  const float R2 = __fmul_rn(R, R);
+  if (!(R2 < 1073741824.0f)) return kRsqCap;
+  return __float2int_rz(R2);
+}
+
+// ---------------------------------------------------------------- 1. footprint
+
+__global__ void footprint_kernel(TileLayout L, int bk, MaskWs ws) {
+  const int nkb = (L.F * L.H * L.W + bk - 1) / bk;
+  const int kb = blockIdx.x * blockDim.x + threadIdx.x;
+  if (kb >= nkb) return;
+  const int N = L.F * L.H * L.W;
+  const int p0 = kb * bk, p1 = min(N, p0 + bk);
+  uint2* rows = ws.rows + static_cast<size_t>(kb) * bk;
+  int4* segs = ws.segs + static_cast<size_t>(kb) * kMaxSeg;
+  int nrows = 0, nseg = 0;
+  int st[kMaxSeg], sylo[kMaxSeg], syhi[kMaxSeg], sxlo[kMaxSeg], sxhi[kMaxSeg];
+  for (int p = p0; p < p1; ++p) {
+    const Coord c = tile_major_coord(L, p);
+    const uint32_t key = (static_cast<uint32_t>(c.t) << 16) | static_cast<uint32_t>(c.y);
+    int f = -1;
+    for (int i = nrows - 1; i >= 0; --i) {
+      if (rows[i].x == key) { f = i; break; }
+    }
+    if (f < 0) {
+      rows[nrows] = make_uint2(key, (static_cast<uint32_t>(c.x) << 16) | static_cast<uint32_t>(c.x));
+      ++nrows;
+    } else {
+      const uint2 rw = rows[f];
+      const int xlo = min(static_cast<int>(rw.y >> 16), c.x);
+      const int xhi = max(static_cast<int>(rw.y & 0xFFFFu), c.x);
+      rows[f].y = (static_cast<uint32_t>(xlo) << 16) | static_cast<uint32_t>(xhi);
+    }
+    if (nseg >= 0) {
+      int s = -1;
+      for (int i = 0; i < nseg; ++i)
+        if (st[i] == c.t) s = i;
+      if (s < 0) {
+        if (nseg == kMaxSeg) {
+          nseg = -1;
+        } else {
+          s = nseg++;
+          st[s] = c.t; sylo[s] = syhi[s] = c.y; sxlo[s] = sxhi[s] = c.x;
+        }
+      }
+      if (s >= 0) {
+        sylo[s] = min(sylo[s], c.y); syhi[s] = max(syhi[s], c.y);
+        sxlo[s] = min(sxlo[s], c.x); sxhi[s] = max(sxhi[s], c.x);
+      }
+    }
+  }
+  // Row-contiguity check: every row's span must be fully covered.
+  int span = 0;
+  for (int i = 0; i < nrows; ++i) {
+    const uint2 rw = rows[i];
+    span += static_cast<int>(rw.y & 0xFFFFu) - static_cast<int>(rw.y >> 16) + 1;
+  }
+  const int tokens = p1 - p0;
+  for (int i = 0; i < max(nseg, 0); ++i)
+    segs[i] = make_int4(st[i], (sylo[i] << 16) | syhi[i], (sxlo[i] << 16) | sxhi[i], 0);
+  ws.info[kb] = make_int4(span == tokens ? nrows : -1, nseg, tokens, 0);
+}
+
+// -------------------------------------------------------------------- 2. votes
+
+struct QueryInfo {
+  int x, y, t;
+  float r;
+};
+
+// Number of keys of key block `kb` inside the support of query q, or, when
+// `exists` is set, 1 if there is at least one and 0 otherwise.
+__device__ __forceinline__ int count_in_block(const QueryInfo& q, int kb, int bk, int nrows,
+                                              const uint2* __restrict__ rows, const float* s_phi,
+                                              const TileLayout& L, int N, bool exists) {
+  int cnt = 0;
+  if (nrows >= 0) {
+    for (int i = 0; i < nrows; ++i) {
+      const uint2 rw = rows[i];
+      const int t = static_cast<int>(rw.x >> 16);
+      const int y = static_cast<int>(rw.x & 0xFFFFu);
+      const int xlo = static_cast<int>(rw.y >> 16);
+      const int xhi = static_cast<int>(rw.y & 0xFFFFu);
+      const int dt = t > q.t ? t - q.t : q.t - t;
+      const int rsq = radius_sq(q.r, s_phi[dt]);
+      const int dy = y - q.y;
+      const int m = rsq - dy * dy;
+      if (m < 0) continue;
+      if (exists) {
+        const int dx = max(0, max(xlo - q.x, q.x - xhi));
+        if (dx * dx <= m) return 1;
+      } else {
+        const int s = isqrt_floor(m);
+        const int lo = max(xlo, q.x - s), hi = min(xhi, q.x + s);
+        if (hi >= lo) cnt += hi - lo + 1;
+      }
+    }
+  } else {
+    const int p1 = min(N, (kb + 1) * bk);
+    for (int p = kb * bk; p < p1; ++p) {
+      const Coord c = tile_major_coord(L, p);
+      const int dt = c.t > q.t ? c.t - q.t : q.t - c.t;
+      const int rsq = radius_sq(q.r, s_phi[dt]);
+      const int dx = c.x - q.x, dy = c.y - q.y;
+      if (dx * dx + dy * dy <= rsq) {
+        if (exists) return 1;
+        ++cnt;
+      }
+    }
+  }
+  return cnt;
+}
+
+// grid (nqb, heads), kVoteThreads threads.  Dynamic smem: 4*F ints (per-frame
+// union boxes of the disks).
+__global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __restrict__ r,
+                                                             const float* __restrict__ phi,
+                                                             TileLayout L, int bq, int bk, int vote,
+                                                             MaskWs ws) {
+  extern __shared__ int s_box[];  // [4][F]: x_lo, x_hi, y_lo, y_hi
+  __shared__ float s_phi[kMaxFrames];
+  __shared__ QueryInfo s_q[128];
+  __shared__ int s_count;
+  const int N = L.F * L.H * L.W;
+  const MaskDims md = mask_dims(L, bq, bk);
+  const int qb = blockIdx.x, h = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int F = L.F;
+  int* bxlo = s_box;
+  int* bxhi = s_box + F;
+  int* bylo = s_box + 2 * F;
+  int* byhi = s_box + 3 * F;
+
+  for (int t = tid; t < F; t += kVoteThreads) {
+    s_phi[t] = phi[t];
+    bxlo[t] = INT_MAX; bxhi[t] = INT_MIN; bylo[t] = INT_MAX; byhi[t] = INT_MIN;
+  }
+  if (tid == 0) s_count = 0;
+  const int q0 = qb * bq;
+  const int nq = min(bq, N - q0);
+  if (tid < nq) {
+    const Coord c = tile_major_coord(L, q0 + tid);
+    float rv = r[static_cast<size_t>(h) * N + q0 + tid];
+    if (rv != rv) rv = __int_as_float(0x7f800000);  // NaN keeps every key, like +inf
+    s_q[tid] = QueryInfo{c.x, c.y, c.t, rv};
+  }
+  __syncthreads();
+
+  // Per key frame: box containing every query's disk in that frame.
+  for (int t = 0; t < F; ++t) {
+    int xlo = INT_MAX, xhi = INT_MIN, ylo = INT_MAX, yhi = INT_MIN;
+    if (tid < nq) {
+      const QueryInfo q = s_q[tid];
+      const int dt = t > q.t ? t - q.t : q.t - t;
+      const int s = isqrt_floor(radius_sq(q.r, s_phi[dt]));
+      xlo = q.x - s; xhi = q.x + s; ylo = q.y - s; yhi = q.y + s;
+    }
+    xlo = __reduce_min_sync(0xffffffffu, xlo);
+    xhi = __reduce_max_sync(0xffffffffu, xhi);
+    ylo = __reduce_min_sync(0xffffffffu, ylo);
+    yhi = __reduce_max_sync(0xffffffffu, yhi);
+    if (lane == 0 && xlo != INT_MAX) {
+      atomicMin(&bxlo[t], xlo); atomicMax(&bxhi[t], xhi);
+      atomicMin(&bylo[t], ylo); atomicMax(&byhi[t], yhi);
+    }
+  }
+  __syncthreads();
+
+  const bool exists = (vote == 1);
+  uint32_t* bits_row = ws.bits + (static_cast<size_t>(h) * md.nqb + qb) * md.nkbw;
+  int my_count = 0;
+  for (int w = warp; w < md.nkbw; w += kVoteThreads / 32) {
+    // prune, lanes over key blocks
+    const int kb = w * 32 + lane;
+    bool survive = false;
+    int4 info = make_int4(0, 0, 0, 0);
+    if (kb < md.nkb) {
+      info = ws.info[kb];
+      if (info.y < 0) {
+        survive = true;
+      } else {
+        const int4* sg = ws.segs + static_cast<size_t>(kb) * kMaxSeg;
+        for (int i = 0; i < info.y && !survive; ++i) {
+          const int4 s = sg[i];
+          const int ylo = s.y >> 16, yhi = s.y & 0xFFFF, xlo = s.z >> 16, xhi = s.z & 0xFFFF;
+          survive = ylo <= byhi[s.x] && yhi >= bylo[s.x] && xlo <= bxhi[s.x] && xhi >= bxlo[s.x];
+        }
+      }
+    }
+    uint32_t cand = __ballot_sync(0xffffffffu, survive);
+    uint32_t word = 0;
+    // exact votes, lanes over queries
+    while (cand) {
+      const int b = __ffs(cand) - 1;
+      cand &= cand - 1;
+      const int kb2 = w * 32 + b;
+      const int nrows = __shfl_sync(0xffffffffu, info.x, b);
+      const uint2* rows = ws.rows + static_cast<size_t>(kb2) * bk;
+      int votes = 0;
+      for (int base = 0; base < nq; base += 32) {
+        const int i = base + lane;
+        int c = 0;
+        if (i < nq) c = count_in_block(s_q[i], kb2, bk, nrows, rows, s_phi, L, N, exists);
+        votes += __reduce_add_sync(0xffffffffu, c);
+        if (votes >= vote) break;
+      }
+      if (votes >= vote) word |= 1u << b;
+    }
+    if (lane == 0) bits_row[w] = word;
+    my_count += __popc(word);
+  }
+  if (lane == 0) atomicAdd(&s_count, my_count);
+  __syncthreads();
+  if (tid == 0) ws.counts[static_cast<size_t>(h) * md.nqb + qb] = s_count;
+}
+
+// --------------------------------------------------------------------- 3. scan
+
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(int heads, int nqb, MaskWs ws,
+                                                            int* row_ptr, int* nnz) {
+  __shared__ long long s_warp[kScanThreads / 32];
+  const long long M = static_cast<long long>(heads) * nqb;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long per = (M + kScanThreads - 1) / kScanThreads;
+  const long long b = tid * per, e = min(M, b + per);
+  long long local = 0;
+  for (long long i = b; i < e; ++i) local += ws.counts[i];
+  // block exclusive scan of `local`
+  long long incl = local;
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    long long v = s_warp[lane];
+    long long vi = v;
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long u = __shfl_up_sync(0xffffffffu, vi, o);
+      if (lane >= o) vi += u;
+    }
+    s_warp[lane] = vi - v;  // exclusive over warps
+  }
+  __syncthreads();
+  long long run = s_warp[warp] + incl - local;
+  for (long long i = b; i < e; ++i) {
+    const int h = static_cast<int>(i / nqb);
+    const int qb = static_cast<int>(i - static_cast<long long>(h) * nqb);
+    row_ptr[static_cast<size_t>(h) * (nqb + 1) + qb] = static_cast<int>(run);
+    run += ws.counts[i];
+    if (qb == nqb - 1) row_ptr[static_cast<size_t>(h) * (nqb + 1) + nqb] = static_cast<int>(run);
+  }
+  if (e == M && b < e) *nnz = static_cast<int>(run);
+  if (M == 0 && tid == 0) *nnz = 0;
+}
+
+// ------------------------------------------------------------------ 4. compact
+
+constexpr int kCompactWarps = 8;
+
+__global__ void __launch_bounds__(kCompactWarps * 32) compact_kernel(int heads, int nqb, int nkbw,
+                                                                     MaskWs ws,
+                                                                     const int* __restrict__ row_ptr,
+                                                                     int* col_idx,
+                                                                     long long capacity) {
+  const int lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * kCompactWarps + (threadIdx.x >> 5);
+  if (row >= static_cast<long long>(heads) * nqb) return;
+  const int h = static_cast<int>(row / nqb);
+  const int qb = static_cast<int>(row - static_cast<long long>(h) * nqb);
+  long long off = row_ptr[static_cast<size_t>(h) * (nqb + 1) + qb];
+  const uint32_t* bits = ws.bits + row * nkbw;
+  for (int base = 0; base < nkbw; base += 32) {
+    const int w = base + lane;
+    uint32_t word = w < nkbw ? bits[w] : 0u;
+    const int c = __popc(word);
+    int incl = c;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    long long pos = off + incl - c;
+    while (word) {
+      const int bit = __ffs(word) - 1;
+      word &= word - 1;
+      if (pos < capacity) col_idx[pos] = w * 32 + bit;
+      ++pos;
+    }
+    off += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+}  // namespace
+
+size_t mask_workspace_bytes(int heads, const TileLayout& L, int block_q, int block_k) {
+  return carve(L, heads, block_q, block_k, nullptr, nullptr);
+}
+
+cudaError_t launch_block_mask(const float* r, const float* phi, int heads, const TileLayout& L,
+                              int block_q, int block_k, int vote, int* row_ptr, int* col_idx,
+                              long long capacity, int* nnz, void* workspace, cudaStream_t stream) {
+  MaskWs ws;
+  carve(L, heads, block_q, block_k, static_cast<char*>(workspace), &ws);
+  const MaskDims md = mask_dims(L, block_q, block_k);
+  footprint_kernel<<<(md.nkb + 127) / 128, 128, 0, stream>>>(L, block_k, ws);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  votes_kernel<<<dim3(md.nqb, heads), kVoteThreads, 4 * L.F * sizeof(int), stream>>>(
+      r, phi, L, block_q, block_k, vote, ws);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  scan_kernel<<<1, kScanThreads, 0, stream>>>(heads, md.nqb, ws, row_ptr, nnz);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long rows = static_cast<long long>(heads) * md.nqb;
+  compact_kernel<<<static_cast<unsigned>((rows + kCompactWarps - 1) / kCompactWarps),
+                   kCompactWarps * 32, 0, stream>>>(heads, md.nqb, md.nkbw, ws, row_ptr, col_idx,
+                                                    capacity);
+  return cudaGetLastError();
+}
+
+}  // namespace tra

@@ -1,0 +1,55 @@
+// Host-side interface between the C ABI (api.cu) and the kernel files.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "tra.h"
+#include "layout.cuh"
+
+namespace tra {
+
+constexpr int kMaxFrames = 1024;   // phi / frame tables live in kernel parameters
+constexpr int kMaxSide = 16384;    // H, W bound: squared distances stay below 2^30
+
+// Device error word of the current device (a module-scope __device__ int).
+int* device_error_word();
+
+// permute.cu
+cudaError_t launch_permute(const void* src, void* dst, tra_dtype in_dtype, tra_dtype out_dtype,
+                           int heads, int d, const TileLayout& L, bool inverse,
+                           cudaStream_t stream);
+
+// radius.cu
+struct FrameTables {
+  float coef[kMaxFrames];  // sqrt(tau / (pi * S(t))) per query frame t
+  float phi[kMaxFrames];   // exp(-gamma * delta)
+};
+cudaError_t launch_budget_radius(const float* H, float* r, float* phi_out, int heads,
+                                 const TileLayout& L, const FrameTables& tables,
+                                 cudaStream_t stream);
+
+// mask.cu
+size_t mask_workspace_bytes(int heads, const TileLayout& L, int block_q, int block_k);
+cudaError_t launch_block_mask(const float* r, const float* phi, int heads, const TileLayout& L,
+                              int block_q, int block_k, int vote, int* row_ptr, int* col_idx,
+                              long long capacity, int* nnz, void* workspace, cudaStream_t stream);
+
+// attention.cu
+struct AttnArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  void* O;
+  float* H;    // entropy (dense only), may be null
+  float* lse;  // may be null
+  const int* row_ptr;  // sparse only
+  const int* col_idx;  // sparse only
+  int heads, N, d;
+  int block_q, block_k;  // sparse only; dense uses 128-key tiles
+  float scale;
+  bool dense;
+};
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream);
+
+}  // namespace tra

@@ -1,0 +1,203 @@
+"""ctypes binding of libtra.so, the C ABI declared in include/tra.h.
+
+Argument marshalling only: every function takes torch tensors that already
+live on the GPU, passes their device pointers, sizes and the current CUDA
+stream to the C entry point of the same name, and raises TraError when the
+call returns a non-zero status.  Nothing here computes any part of the
+method, and there is no fallback: if libtra.so is missing the first call
+raises.
+"""
+import ctypes
+import math
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtra.so")
+
+TRA_BF16, TRA_F32 = 0, 1
+STATUS = {0: "TRA_OK", 1: "TRA_ERR_INVALID_ARGUMENT", 2: "TRA_ERR_UNSUPPORTED",
+          3: "TRA_ERR_WORKSPACE", 4: "TRA_ERR_CAPACITY", 5: "TRA_ERR_CUDA",
+          6: "TRA_ERR_DEVICE", 7: "TRA_ERR_TIMEOUT"}
+
+
+class TraError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn}: {STATUS.get(status, status)} ({text})")
+        self.status = status
+
+
+class Grid(ctypes.Structure):
+    _fields_ = [("F", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int)]
+
+
+class Tile(ctypes.Structure):
+    _fields_ = [("t", ctypes.c_int), ("y", ctypes.c_int), ("x", ctypes.c_int)]
+
+
+_lib = None
+_c_int, _c_ll, _c_size, _c_float, _vp = (ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t,
+                                         ctypes.c_float, ctypes.c_void_p)
+
+_PROTOS = {
+    "tra_status_string": (ctypes.c_char_p, [_c_int]),
+    "tra_version": (_c_int, []),
+    "tra_tile_major_permute": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, Grid, Tile, _vp]),
+    "tra_inverse_permute": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, Grid, Tile, _vp]),
+    "tra_dense_attn_entropy": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
+                                        _c_float, _vp]),
+    "tra_budget_radius": (_c_int, [_vp, _vp, _vp, _c_int, Grid, Tile, _c_float, _c_float, _vp]),
+    "tra_mask_workspace_size": (_c_size, [_c_int, Grid, Tile, _c_int, _c_int]),
+    "tra_build_block_mask": (_c_int, [_vp, _vp, _c_int, Grid, Tile, _c_int, _c_int, _c_int, _vp,
+                                      _vp, _c_ll, _vp, _vp, _c_size, _vp]),
+    "tra_block_sparse_attn": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
+                                       _c_int, _c_int, _c_float, _vp]),
+    "tra_get_device_error": (_c_int, [ctypes.POINTER(_c_int), _vp]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libtra.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m entropy_adaptive_radius_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _PROTOS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().tra_status_string(s).decode()
+
+
+def _check(fn: str, s: int):
+    if s != 0:
+        raise TraError(fn, s, status_string(s))
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return TRA_BF16
+    if t.dtype == torch.float32:
+        return TRA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _grid(grid: Sequence[int]) -> Grid:
+    return Grid(*map(int, grid))
+
+
+def _tile(tile: Sequence[int]) -> Tile:
+    return Tile(*map(int, tile))
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def tra_tile_major_permute(X, X_tm, grid, tile=(1, 4, 4), stream=None):
+    """X_tm[h, p] = X[h, pi(p)] for X [heads, N, d] (bf16 or f32)."""
+    _contig(X, X_tm)
+    heads, _, d = X.shape
+    _check("tra_tile_major_permute", lib().tra_tile_major_permute(
+        _p(X), _p(X_tm), _dtype(X), _dtype(X_tm), heads, d, _grid(grid), _tile(tile),
+        _stream(stream)))
+    return X_tm
+
+
+def tra_inverse_permute(X_tm, X, grid, tile=(1, 4, 4), stream=None):
+    """X[h, pi(p)] = X_tm[h, p]."""
+    _contig(X, X_tm)
+    if X.dtype != X_tm.dtype:
+        raise TypeError("inverse permute keeps the dtype")
+    heads, _, d = X_tm.shape
+    _check("tra_inverse_permute", lib().tra_inverse_permute(
+        _p(X_tm), _p(X), _dtype(X_tm), heads, d, _grid(grid), _tile(tile), _stream(stream)))
+    return X
+
+
+def tra_dense_attn_entropy(Q, K, V, O, H, lse=None, scale=None, stream=None):
+    """Dense attention O, entropy H and (optionally) LSE of Q, K, V [heads, N, d] bf16."""
+    _contig(Q, K, V, O, H, lse)
+    heads, N, d = Q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    _check("tra_dense_attn_entropy", lib().tra_dense_attn_entropy(
+        _p(Q), _p(K), _p(V), _p(O), _p(H), _p(lse), heads, N, d, scale, _stream(stream)))
+    return O, H
+
+
+def tra_budget_radius(H, r, grid, tau, gamma, tile=(1, 4, 4), phi_out=None, stream=None):
+    """Per-query base radius r [heads, N] from entropy H (tile-major order)."""
+    _contig(H, r, phi_out)
+    heads = H.shape[0]
+    _check("tra_budget_radius", lib().tra_budget_radius(
+        _p(H), _p(r), _p(phi_out), heads, _grid(grid), _tile(tile), float(tau), float(gamma),
+        _stream(stream)))
+    return r
+
+
+def tra_mask_workspace_size(heads, grid, block_q, block_k, tile=(1, 4, 4)) -> int:
+    return int(lib().tra_mask_workspace_size(heads, _grid(grid), _tile(tile), block_q, block_k))
+
+
+def tra_build_block_mask(r, phi, grid, block_q, block_k, vote, row_ptr, col_idx, nnz, workspace,
+                         tile=(1, 4, 4), stream=None):
+    """Block-sparse CSR of the radius mask.  `workspace` is a uint8 CUDA tensor of
+    at least tra_mask_workspace_size bytes (256-byte aligned)."""
+    _contig(r, phi, row_ptr, col_idx, nnz, workspace)
+    heads = r.shape[0]
+    _check("tra_build_block_mask", lib().tra_build_block_mask(
+        _p(r), _p(phi), heads, _grid(grid), _tile(tile), block_q, block_k, vote, _p(row_ptr),
+        _p(col_idx), col_idx.numel(), _p(nnz), _p(workspace), workspace.numel(),
+        _stream(stream)))
+    return row_ptr, col_idx, nnz
+
+
+def tra_block_sparse_attn(Q, K, V, O, row_ptr, col_idx, block_q, block_k, lse=None, scale=None,
+                          stream=None):
+    """Exact attention over the kept blocks of the CSR mask."""
+    _contig(Q, K, V, O, row_ptr, col_idx, lse)
+    heads, N, d = Q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    _check("tra_block_sparse_attn", lib().tra_block_sparse_attn(
+        _p(Q), _p(K), _p(V), _p(O), _p(lse), _p(row_ptr), _p(col_idx), heads, N, d, block_q,
+        block_k, scale, _stream(stream)))
+    return O
+
+
+def tra_get_device_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error code."""
+    code = _c_int(0)
+    s = lib().tra_get_device_error(ctypes.byref(code), _stream(stream))
+    if s not in (0, 7):
+        _check("tra_get_device_error", s)
+    return code.value
+
+
+def workspace_tensor(nbytes: int, device="cuda") -> torch.Tensor:
+    """A uint8 CUDA buffer of `nbytes` whose start is 256-byte aligned (torch's
+    caching allocator returns 512-byte aligned blocks)."""
+    t = torch.empty(max(1, nbytes), dtype=torch.uint8, device=device)
+    if t.data_ptr() % 256:
+        raise RuntimeError("allocator returned a misaligned workspace")
+    return t

@@ -1,0 +1,208 @@
+/*
+ * tra.h — C ABI of the Token Radius Attention (TRA) hot path on B200 (sm_100a).
+ *
+ * The method: "Token Radius Attention for Efficient Video Generation"
+ * (summaries at gist.science, paper 2608.02504; section names below follow
+ * those pages).  A dense warm-up attention pass also yields every query's
+ * softmax entropy H_i; the entropy sets a per-query token budget
+ * B_i = tau * exp(H_i) / N (§2 Insight I); the budget becomes a base radius
+ * that shrinks with temporal distance by phi(delta) = exp(-gamma * delta)
+ * (§2 Insight II); a fused kernel turns the per-token disks into a
+ * block-sparse query-block x key-block mask over a tile-major token order
+ * (§2 "TRA pipeline", efficient execution); later denoising steps run exact
+ * softmax attention over the kept blocks only, reusing the entropy
+ * (cross-step reuse).
+ *
+ * Conventions shared by every call:
+ *  - Pointers are DEVICE pointers owned by the caller unless a comment says
+ *    otherwise.  The library never allocates device memory; scratch space is
+ *    passed in (see tra_mask_workspace_size).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and never synchronises, except tra_get_device_error.
+ *  - Every call checks its arguments first and launches nothing when it
+ *    returns an error.  heads == 0 or N == 0 is a valid empty problem.
+ *  - Tensors are [heads, N, d] with d contiguous (batch folded into heads),
+ *    N = F * H * W tokens.  The original token order is (t, y, x) row-major,
+ *    token n = (t * H + y) * W + x.
+ *  - Calls on distinct streams may run concurrently from several threads.
+ *  - A device-side wait that runs out of time (it never should) makes the
+ *    kernel record a code in a device error word and return early; the next
+ *    tra_get_device_error reports it.  No kernel traps.
+ *  - Requires a compute capability 10.0 GPU (B200, sm_100a).
+ */
+#ifndef TRA_H_
+#define TRA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* tra_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  TRA_OK = 0,
+  TRA_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misaligned pointer */
+  TRA_ERR_UNSUPPORTED = 2,      /* valid but outside the supported shapes */
+  TRA_ERR_WORKSPACE = 3,        /* workspace too small or misaligned */
+  TRA_ERR_CAPACITY = 4,         /* col_idx capacity negative */
+  TRA_ERR_CUDA = 5,             /* a CUDA runtime call failed (launch, attribute) */
+  TRA_ERR_DEVICE = 6,           /* no usable sm_100 device */
+  TRA_ERR_TIMEOUT = 7           /* reported by tra_get_device_error */
+} tra_status;
+
+typedef enum { TRA_BF16 = 0, TRA_F32 = 1 } tra_dtype;
+
+/* Latent video grid: F frames of H x W tokens. */
+typedef struct { int F, H, W; } tra_grid;
+
+/* Tile shape of the tile-major order: t frames x y rows x x columns. */
+typedef struct { int t, y, x; } tra_tile;
+
+/* Static description of a status code; never NULL. */
+const char* tra_status_string(tra_status s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int tra_version(void);
+
+/*
+ * Tile-major permutation (§2 "TRA pipeline", tile-major layout: tokens are
+ * re-ordered so that spatial neighbours are contiguous).
+ *
+ * X_tm[h, p, :] = X[h, pi(p), :], where pi walks the tiles of `tile` in
+ * (frame-tile, tile-row, tile-col) order and, inside a tile, its tokens in
+ * (t, y, x) row-major order; tiles at the grid's far edges are truncated, so
+ * pi is a bijection on [0, N).
+ *   X     [heads, N, d] of in_dtype, original order; read only.
+ *   X_tm  [heads, N, d] of out_dtype, tile-major order; written.  Must not
+ *         overlap X.  f32 -> bf16 rounds to nearest even.
+ *   d     multiple of 8, 8..1024.  X and X_tm 16-byte aligned.
+ */
+tra_status tra_tile_major_permute(const void* X, void* X_tm, tra_dtype in_dtype,
+                                  tra_dtype out_dtype, int heads, int d, tra_grid grid,
+                                  tra_tile tile, tra_stream_t stream);
+
+/*
+ * Inverse of tra_tile_major_permute: X[h, pi(p), :] = X_tm[h, p, :].
+ * Same dtype on both sides; same shape rules.
+ */
+tra_status tra_inverse_permute(const void* X_tm, void* X, tra_dtype dtype, int heads, int d,
+                               tra_grid grid, tra_tile tile, tra_stream_t stream);
+
+/*
+ * Dense warm-up attention with per-query entropy (§2 "TRA pipeline" step 1:
+ * entropy of every query from the dense warm-up phase; §3 contribution 3:
+ * fused entropy kernel).
+ *
+ * For every head and query i (rows of Q, any fixed token order):
+ *   s_ij = scale * q_i . k_j over all N keys j,
+ *   O_i  = sum_j softmax(s_i)_j v_j                 (bf16, fp32 accumulation)
+ *   H_i  = ln Z_i - (sum_j e^{s_ij} s_ij) / Z_i,  Z_i = sum_j e^{s_ij}
+ *                                                 (natural log, fp32)
+ *   lse_i = ln Z_i                                 (fp32; optional)
+ *   Q, K, V  [heads, N, d] bf16, 16-byte aligned; read only.
+ *   O        [heads, N, d] bf16; written.
+ *   H        [heads, N] fp32; written.
+ *   lse      [heads, N] fp32 or NULL.
+ *   d        64 or 128.   scale > 0 and finite (1/sqrt(d) for standard SDPA).
+ *   N        1 .. 2^24 (0 is an empty problem).
+ * Tensor cores (tcgen05, bf16 in, fp32 accumulators in tensor memory) run
+ * QK^T and PV; entropy statistics are kept in fp32 beside the online softmax.
+ */
+tra_status tra_dense_attn_entropy(const void* Q, const void* K, const void* V, void* O,
+                                  float* H, float* lse, int heads, int N, int d, float scale,
+                                  tra_stream_t stream);
+
+/*
+ * Entropy -> budget -> radius (§2 Insight I: B_i = tau * exp(H_i) / N;
+ * Insight II and pipeline step 2: budget -> query-specific base radius,
+ * per-frame radius r_i * phi(|dt|), phi(delta) = exp(-gamma * delta)).
+ *
+ * The budget becomes a radius by equal area: the disks of all key frames
+ * together hold K_i = B_i * N tokens,
+ *   K_i = pi * r_i^2 * S(t_i),   S(t) = sum_{t'=0}^{F-1} phi(|t' - t|)^2,
+ * so r_i = sqrt(tau * exp(H_i) / (pi * S(t_i))), with t_i the frame of query i.
+ *   H        [heads, N] fp32 in TILE-MAJOR order (as produced by the dense
+ *            call on permuted inputs); read only.  +inf gives r = +inf,
+ *            NaN gives NaN (the mask keeps every key for either).
+ *   r        [heads, N] fp32, tile-major order; written.
+ *   phi_out  [F] fp32 or NULL: phi(delta) for delta = 0..F-1, the table the
+ *            mask call reads.  Computed in double on the host, rounded once.
+ *   tau >= 0 and finite; gamma >= 0 and finite; F <= 1024.
+ */
+tra_status tra_budget_radius(const float* H, float* r, float* phi_out, int heads, tra_grid grid,
+                             tra_tile tile, float tau, float gamma, tra_stream_t stream);
+
+/*
+ * Bytes of device scratch space tra_build_block_mask needs for these sizes
+ * (0 if the sizes are invalid).  The space must be 256-byte aligned.
+ */
+size_t tra_mask_workspace_size(int heads, tra_grid grid, tra_tile tile, int block_q, int block_k);
+
+/*
+ * Fused radius mask -> block-sparse CSR (§2 "TRA pipeline", efficient
+ * execution: one kernel fuses distance computation, radius comparison, block
+ * pruning and token voting, turning the irregular token-level radius mask
+ * into a regular block-sparse mask).
+ *
+ * Token mask: key j is in query i's support when
+ *     dx^2 + dy^2 <= R2,   R2 = fl32(R * R),  R = fl32(r_i * phi[|t_j - t_i|])
+ * (integer token distances, inclusive compare, rounded fp32 products with no
+ * fused multiply-add; a radius of +inf or NaN keeps every key).
+ * Blocks are consecutive runs of block_q (block_k) TILE-MAJOR positions, the
+ * last one possibly shorter.  votes(qb, kb) = number of token pairs in the
+ * support with the query in qb and the key in kb; a block pair is kept when
+ * votes >= vote_threshold.  Pruning by per-frame bounding boxes only skips
+ * pairs with no votes, so the mask equals the brute-force definition.
+ *   r            [heads, N] fp32 tile-major; read only.
+ *   phi          [F] fp32 device table (e.g. written by tra_budget_radius).
+ *   row_ptr      [heads * (nqb + 1)] int32, nqb = ceil(N / block_q); written.
+ *                Row (h, qb) is col_idx[row_ptr[h*(nqb+1)+qb] .. row_ptr[h*(nqb+1)+qb+1]);
+ *                offsets are global over all heads (row_ptr[0] = 0).
+ *   col_idx      [col_capacity] int32; written: kept kb of each row, ascending.
+ *   nnz          [1] int32; written: total kept blocks.  If it exceeds
+ *                col_capacity after the call completes, col_idx holds only the
+ *                first col_capacity entries (capacity h*nqb*nkb never overflows).
+ *   workspace    >= tra_mask_workspace_size(...) bytes, 256-byte aligned.
+ *   block_q, block_k in {16, 64, 128};  vote_threshold >= 1;  tile as given
+ *   to tra_tile_major_permute;  F <= 1024;  H, W <= 16384.
+ */
+tra_status tra_build_block_mask(const float* r, const float* phi, int heads, tra_grid grid,
+                                tra_tile tile, int block_q, int block_k, int vote_threshold,
+                                int* row_ptr, int* col_idx, long long col_capacity, int* nnz,
+                                void* workspace, size_t workspace_bytes, tra_stream_t stream);
+
+/*
+ * Block-sparse attention over the kept blocks (§2 "TRA pipeline": the
+ * block-sparse mask drives a block-sparse attention backend; reuse across
+ * sparse steps).  Exact softmax over every token of the kept key blocks of
+ * each query's block row; tokens >= N are excluded; a query whose row keeps
+ * nothing gets O = 0 and lse = -inf.
+ *   Q, K, V   [heads, N, d] bf16 tile-major, 16-byte aligned; read only.
+ *   O         [heads, N, d] bf16; written.
+ *   lse       [heads, N] fp32 natural-log sum of exponentials, or NULL.
+ *   row_ptr, col_idx  CSR as written by tra_build_block_mask for the same
+ *             heads, N, block_q, block_k (col_idx ascending, no repeats).
+ *   d in {64, 128}; block_q, block_k in {16, 64, 128};  when block_q < 128,
+ *   ceil(N / block_k) <= 1024.  scale > 0 and finite.
+ */
+tra_status tra_block_sparse_attn(const void* Q, const void* K, const void* V, void* O,
+                                 float* lse, const int* row_ptr, const int* col_idx, int heads,
+                                 int N, int d, int block_q, int block_k, float scale,
+                                 tra_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  *code = 0 when no kernel recorded an error; otherwise the
+ * code of the first wait that ran out of time.  Returns TRA_ERR_TIMEOUT when
+ * *code != 0, TRA_ERR_CUDA when the stream reported a CUDA error.
+ */
+tra_status tra_get_device_error(int* code, tra_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRA_H_ */

@@ -1,0 +1,133 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry
+point that include/tra.h declares, and rejects bad arguments before touching
+a device (and reports a missing device instead of falling back)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from entropy_adaptive_radius_b200 import build as tra_build
+from entropy_adaptive_radius_b200 import tra
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tra.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE, CAPACITY, CUDA, DEVICE = 0, 1, 2, 3, 4, 5, 6
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(tra.LIB_PATH):
+        tra_build.build(quiet=True)
+    return tra.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tra_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_six_calls():
+    names = declared_functions()
+    for n in ("tra_tile_major_permute", "tra_inverse_permute", "tra_dense_attn_entropy",
+              "tra_budget_radius", "tra_build_block_mask", "tra_block_sparse_attn"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for s in range(8):
+        assert len(tra.status_string(s)) > 0
+    assert tra.status_string(99) == "unknown status"
+    assert L.tra_version() >= 100
+
+
+G = tra.Grid(21, 45, 80)
+T = tra.Tile(1, 4, 4)
+P = ctypes.c_void_p(4096)      # a 16-byte aligned stand-in address, never dereferenced
+P2 = ctypes.c_void_p(8192)
+MIS = ctypes.c_void_p(4104)    # misaligned
+S0 = ctypes.c_void_p(0)
+
+
+def test_permute_validation(L):
+    f = L.tra_tile_major_permute
+    assert f(None, P, 0, 0, 2, 128, G, T, S0) == INVALID
+    assert f(P, None, 0, 0, 2, 128, G, T, S0) == INVALID
+    assert f(MIS, P, 0, 0, 2, 128, G, T, S0) == INVALID
+    assert f(P, P, 0, 0, 2, 128, G, T, S0) == INVALID
+    assert f(P, P2, 5, 0, 2, 128, G, T, S0) == INVALID
+    assert f(P, P2, 0, 0, 2, 100, G, T, S0) == UNSUPPORTED
+    assert f(P, P2, 0, 0, -1, 128, G, T, S0) == INVALID
+    assert f(P, P2, 0, 0, 2, 128, tra.Grid(-1, 2, 2), T, S0) == INVALID
+    assert f(P, P2, 0, 0, 2, 128, G, tra.Tile(0, 4, 4), S0) == INVALID
+    assert f(P, P2, 0, 0, 2, 128, tra.Grid(2000, 2, 2), T, S0) == INVALID   # F > 1024
+    # empty problems are valid no-ops
+    assert f(None, None, 0, 0, 0, 128, G, T, S0) == OK
+    assert f(None, None, 0, 0, 2, 128, tra.Grid(0, 45, 80), T, S0) == OK
+    g = L.tra_inverse_permute
+    assert g(P, P2, 0, 2, 100, G, T, S0) == UNSUPPORTED
+    assert g(P, None, 0, 2, 128, G, T, S0) == INVALID
+
+
+def test_attention_validation(L):
+    d = L.tra_dense_attn_entropy
+    assert d(P, P, P, P, P, None, 2, 1000, 96, 0.1, S0) == UNSUPPORTED
+    assert d(P, P, P, P, P, None, 2, 1000, 128, 0.0, S0) == INVALID
+    assert d(P, P, P, P, P, None, 2, 1000, 128, float("nan"), S0) == INVALID
+    assert d(P, P, P, P, None, None, 2, 1000, 128, 0.1, S0) == INVALID   # H required
+    assert d(P, None, P, P, P, None, 2, 1000, 128, 0.1, S0) == INVALID
+    assert d(P, P, MIS, P, P, None, 2, 1000, 128, 0.1, S0) == INVALID
+    assert d(P, P, P, P, P, None, 0, 1000, 128, 0.1, S0) == OK
+    assert d(P, P, P, P, P, None, 2, 0, 128, 0.1, S0) == OK
+    assert d(P, P, P, P, P, None, 2, (1 << 24) + 1, 128, 0.1, S0) == UNSUPPORTED
+    s = L.tra_block_sparse_attn
+    assert s(P, P, P, P, None, P, P, 2, 1000, 128, 32, 128, 0.1, S0) == UNSUPPORTED
+    assert s(P, P, P, P, None, P, P, 2, 1000, 128, 128, 48, 0.1, S0) == UNSUPPORTED
+    assert s(P, P, P, P, None, None, P, 2, 1000, 128, 128, 128, 0.1, S0) == INVALID
+    # query blocks below 128 rows merge lists of at most 1024 key blocks
+    assert s(P, P, P, P, None, P, P, 2, 64 * 1025, 128, 64, 64, 0.1, S0) == UNSUPPORTED
+
+
+def test_radius_and_mask_validation(L):
+    b = L.tra_budget_radius
+    assert b(P, P, None, 2, G, T, -1.0, 0.3, S0) == INVALID
+    assert b(P, P, None, 2, G, T, 1.0, float("inf"), S0) == INVALID
+    assert b(None, P, None, 2, G, T, 1.0, 0.3, S0) == INVALID
+    assert b(None, None, None, 0, G, T, 1.0, 0.3, S0) == OK
+    m = L.tra_build_block_mask
+    ws = L.tra_mask_workspace_size(40, G, T, 128, 128)
+    assert ws > 0
+    assert m(P, P, 40, G, T, 128, 48, 1, P, P, 100, P, P, ws, S0) == UNSUPPORTED
+    assert m(P, P, 40, G, T, 128, 128, 0, P, P, 100, P, P, ws, S0) == INVALID
+    assert m(P, P, 40, G, T, 128, 128, 1, P, P, -1, P, P, ws, S0) == CAPACITY
+    assert m(P, P, 40, G, T, 128, 128, 1, P, P, 100, None, P, ws, S0) == INVALID
+    assert m(P, P, 40, G, T, 128, 128, 1, P, P, 100, P, P, ws - 1, S0) == WORKSPACE
+    assert m(P, P, 40, G, T, 128, 128, 1, P, P, 100, P, ctypes.c_void_p(4096 + 128), ws, S0) == WORKSPACE
+    assert m(None, P, 40, G, T, 128, 128, 1, P, P, 100, P, P, ws, S0) == INVALID
+
+
+def test_workspace_size_grows_with_problem(L):
+    small = L.tra_mask_workspace_size(2, tra.Grid(4, 8, 8), T, 16, 16)
+    big = L.tra_mask_workspace_size(40, G, T, 128, 128)
+    assert 0 < small < big
+    assert L.tra_mask_workspace_size(2, G, T, 100, 128) == 0
+    # bitmask rows dominate: heads * nqb * ceil(nkb/32) words
+    nqb = -(-75600 // 128)
+    assert big >= 40 * nqb * (-(-nqb // 32)) * 4
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_valid_call_without_gpu_reports_device_error(L):
+    # No silent CPU fallback: a well-formed call on a machine without an
+    # sm_100 GPU returns TRA_ERR_DEVICE and the binding raises.
+    assert L.tra_tile_major_permute(P, P2, 0, 0, 2, 128, G, T, S0) == DEVICE
+    with pytest.raises(tra.TraError):
+        tra._check("x", DEVICE)
