@@ -1,0 +1,598 @@
+"""Benchmark of the Token Radius Attention hot path on B200.
+
+One step = one pass of the whole hot path on the Wan2.1-14B 720p-shaped
+workload (grid 21x45x80, N = 75600 tokens, 40 heads, d = 128, bf16, 128x128
+blocks, gamma = 0.3, vote 1): a dense warm-up call (tile-major permute of Q,
+K, V; dense attention + entropy; entropy -> radius; fused mask -> CSR; inverse
+permute of O), then 4 block-sparse calls that reuse the warm-up's CSR on
+perturbed Q/K (permute, block-sparse attention, inverse permute).  tau is
+calibrated once (outside the timed region) so that ~12% of the blocks are kept.
+
+`value` is the step's attention work on kept blocks (4*d*|qb|*|kb| flops per
+kept block pair; the dense call keeps every pair) divided by the step time,
+measured with CUDA events, inputs resident in HBM (each input tensor is
+774 MB, larger than the 126 MB L2).  Per-kernel times come from CUDA events
+around each launch on the launching stream.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun every rank runs its own independent workload (weak scaling:
+different inputs, same shape; no collective on the data path).
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from entropy_adaptive_radius_b200 import inputs, workloads  # noqa: E402
+
+METRIC = "block-sparse TRA attention ms/call & TFLOP/s (kept blocks) at 1 B200; mask ms"
+UNIT = "TFLOP/s"
+WL = workloads.WAN14B
+
+
+# --------------------------------------------------------------------- helpers
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index, path):
+        self.index, self.path, self.proc = index, path, None
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons)}
+        # median over the samples taken under load (top 80% of the clock samples)
+        sm_sorted = sorted(sm)
+        loaded = sm_sorted[len(sm_sorted) // 5:] or sm_sorted
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kept_pair_tokens(row_ptr, col_idx, heads, N, bq, bk):
+    """sum over kept (qb, kb) of |qb| * |kb| (tail blocks shorter), all heads."""
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    rp = row_ptr.reshape(heads, nqb + 1)
+    qsz = np.minimum(bq, N - np.arange(nqb) * bq).astype(np.int64)
+    ksz = np.minimum(bk, N - np.arange(nkb) * bk).astype(np.int64)
+    total = 0
+    for h in range(heads):
+        s, e = int(rp[h, 0]), int(rp[h, nqb])
+        cols = col_idx[s:e]
+        counts = np.diff(rp[h])
+        rows = np.repeat(np.arange(nqb), counts)
+        total += int((qsz[rows] * ksz[cols]).sum())
+    return total
+
+
+# ------------------------------------------------------------------- GPU arm
+
+class Pipeline:
+    """Device buffers and launches of one TRA layer (all calls through the C ABI)."""
+
+    def __init__(self, wl, device):
+        from entropy_adaptive_radius_b200 import tra
+        self.tra = tra
+        self.wl = wl
+        self.grid = (wl.F, wl.H, wl.W)
+        h, N, d = wl.heads, wl.N, wl.d
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.Qtm, self.Ktm, self.Vtm = (torch.empty(h, N, d, **bf) for _ in range(3))
+        self.Otm = torch.empty(h, N, d, **bf)
+        self.O = torch.empty(h, N, d, **bf)
+        self.H = torch.empty(h, N, dtype=torch.float32, device=device)
+        self.r = torch.empty_like(self.H)
+        self.phi = torch.empty(wl.F, dtype=torch.float32, device=device)
+        self.nqb, self.nkb = wl.nqb, wl.nkb
+        self.row_ptr = torch.empty(h * (self.nqb + 1), dtype=torch.int32, device=device)
+        self.col_idx = torch.empty(h * self.nqb * self.nkb, dtype=torch.int32, device=device)
+        self.nnz = torch.empty(1, dtype=torch.int32, device=device)
+        self.ws = tra.workspace_tensor(
+            tra.tra_mask_workspace_size(h, self.grid, wl.block_q, wl.block_k, wl.tile), device)
+        self.launches = 0
+        self.tau = 1.0
+
+    def mask(self, tau):
+        w, t = self.wl, self.tra
+        t.tra_budget_radius(self.H, self.r, self.grid, tau, w.gamma, w.tile, phi_out=self.phi)
+        t.tra_build_block_mask(self.r, self.phi, self.grid, w.block_q, w.block_k, w.vote,
+                               self.row_ptr, self.col_idx, self.nnz, self.ws, w.tile)
+        self.launches += 5
+
+    def warmup_call(self, Q, K, V, rec):
+        t = self.tra
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        e[0].record()
+        for X, Y in ((Q, self.Qtm), (K, self.Ktm), (V, self.Vtm)):
+            t.tra_tile_major_permute(X, Y, self.grid, self.wl.tile)
+        e[1].record()
+        t.tra_dense_attn_entropy(self.Qtm, self.Ktm, self.Vtm, self.Otm, self.H)
+        e[2].record()
+        t.tra_budget_radius(self.H, self.r, self.grid, self.tau, self.wl.gamma, self.wl.tile,
+                            phi_out=self.phi)
+        e[3].record()
+        t.tra_build_block_mask(self.r, self.phi, self.grid, self.wl.block_q, self.wl.block_k,
+                               self.wl.vote, self.row_ptr, self.col_idx, self.nnz, self.ws,
+                               self.wl.tile)
+        e[4].record()
+        t.tra_inverse_permute(self.Otm, self.O, self.grid, self.wl.tile)
+        e[5].record()
+        self.launches += 3 + 1 + 1 + 4 + 1
+        if rec is not None:
+            rec.append(("warmup", e))
+
+    def sparse_call(self, Q, K, V, rec):
+        t = self.tra
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record()
+        for X, Y in ((Q, self.Qtm), (K, self.Ktm), (V, self.Vtm)):
+            t.tra_tile_major_permute(X, Y, self.grid, self.wl.tile)
+        e[1].record()
+        t.tra_block_sparse_attn(self.Qtm, self.Ktm, self.Vtm, self.Otm, self.row_ptr,
+                                self.col_idx, self.wl.block_q, self.wl.block_k)
+        e[2].record()
+        t.tra_inverse_permute(self.Otm, self.O, self.grid, self.wl.tile)
+        e[3].record()
+        self.launches += 5
+        if rec is not None:
+            rec.append(("sparse", e))
+
+    def kept_fraction(self):
+        return int(self.nnz.item()) / (self.wl.heads * self.nqb * self.nkb)
+
+
+def calibrate_tau(pipe, target, log):
+    """Bisection of log(tau) on the kept-block fraction (monotone in tau)."""
+    lo, hi = math.log(1e-6), math.log(1e4)
+    best = None
+    for _ in range(30):
+        mid = 0.5 * (lo + hi)
+        pipe.mask(math.exp(mid))
+        f = pipe.kept_fraction()
+        if best is None or abs(f - target) < abs(best[1] - target):
+            best = (math.exp(mid), f)
+        if abs(f - target) < 0.002:
+            break
+        if f > target:
+            hi = mid
+        else:
+            lo = mid
+    log(f"tau calibrated: tau={best[0]:.5g} kept={best[1]:.4f} (target {target})")
+    return best[0]
+
+
+def gpu_arm(args, rank, world, local):
+    import torch.distributed as dist
+    from entropy_adaptive_radius_b200 import tra
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    log = (lambda m: print(f"[bench] {m}", file=sys.stderr, flush=True)) if rank == 0 else (lambda m: None)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=device,
+                                timeout=__import__("datetime").timedelta(seconds=600))
+    wl = WL
+    calls = wl.sparse_calls
+    t0 = time.time()
+    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed, wl.q_scale, "bf16",
+                              head_offset=rank * wl.heads)
+    pert = [(inputs.perturb(Q, wl.seed, c, 0, head_offset=rank * wl.heads),
+             inputs.perturb(K, wl.seed, c, 1, head_offset=rank * wl.heads)) for c in range(1, calls + 1)]
+    log(f"inputs generated in {time.time() - t0:.1f}s")
+    host = [Q, K, V] + [x for qk in pert for x in qk]
+    host = [x.pin_memory() for x in host]
+    dev = [x.to(device) for x in host]
+    Qd, Kd, Vd = dev[0], dev[1], dev[2]
+    sparse_in = [(dev[3 + 2 * i], dev[4 + 2 * i], Vd) for i in range(calls)]
+
+    pipe = Pipeline(wl, device)
+    # dense warm-up once to get H, then calibrate tau on it
+    pipe.warmup_call(Qd, Kd, Vd, None)
+    torch.cuda.synchronize()
+    pipe.tau = calibrate_tau(pipe, wl.kept_target, log)
+    pipe.warmup_call(Qd, Kd, Vd, None)
+    torch.cuda.synchronize()
+    kept = pipe.kept_fraction()
+    rp = pipe.row_ptr.cpu().numpy()
+    ci = pipe.col_idx[: int(pipe.nnz.item())].cpu().numpy()
+    kept_pairs = kept_pair_tokens(rp, ci, wl.heads, wl.N, wl.block_q, wl.block_k)
+    fl_sparse = 4.0 * wl.d * kept_pairs                  # per sparse call
+    fl_dense = 4.0 * wl.d * wl.N * wl.N * wl.heads      # the warm-up keeps every pair
+    fl_step = fl_dense + calls * fl_sparse
+
+    def step(rec):
+        pipe.warmup_call(Qd, Kd, Vd, rec)
+        for c in range(calls):
+            pipe.sparse_call(*sparse_in[c], rec)
+
+    for _ in range(args.warmup):
+        step(None)
+    torch.cuda.synchronize()
+    if tra.tra_get_device_error() != 0:
+        raise RuntimeError("device-side wait timed out during warm-up")
+
+    sampler = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+                           if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/tra_clocks_{rank}.csv")
+    rec = []
+    pipe.launches = 0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("timed")
+    start.record()
+    for _ in range(args.steps):
+        step(rec)
+    stop.record()
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    elapsed_ms = start.elapsed_time(stop)
+    launches = pipe.launches
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+        dist.barrier()
+    if tra.tra_get_device_error() != 0:
+        raise RuntimeError("device-side wait timed out in the timed region")
+
+    # per-kernel times (launching stream = current stream)
+    dense_ms, sparse_ms, mask_ms, radius_ms, perm_ms = [], [], [], [], []
+    for kind, e in rec:
+        if kind == "warmup":
+            perm_ms.append(e[0].elapsed_time(e[1]) + e[4].elapsed_time(e[5]))
+            dense_ms.append(e[1].elapsed_time(e[2]))
+            radius_ms.append(e[2].elapsed_time(e[3]))
+            mask_ms.append(e[3].elapsed_time(e[4]))
+        else:
+            perm_ms.append(e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]))
+            sparse_ms.append(e[1].elapsed_time(e[2]))
+    ms_step = elapsed_ms / args.steps
+    value = world * fl_step / (ms_step * 1e-3) / 1e12
+    d_ms, s_ms = statistics.mean(dense_ms), statistics.mean(sparse_ms)
+    peaks, peak_kind = load_peaks()
+    dense_tf = fl_dense / (d_ms * 1e-3) / 1e12
+    sparse_tf = fl_sparse / (s_ms * 1e-3) / 1e12
+    # dominant kernel of the step by device time
+    dense_total, sparse_total = d_ms, calls * s_ms
+    dom = ("dense_attn_entropy", dense_tf) if dense_total >= sparse_total else ("block_sparse_attn", sparse_tf)
+    peak_sus = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    roofline = {"kernel": dom[0], "bound": "tensor", "achieved": round(dom[1], 2),
+                "peak": peak_sus, "unit": "TFLOP/s", "frac": round(dom[1] / peak_sus, 4),
+                "traffic": None, "peak_kind": f"{peak_kind} bf16 sustained"}
+    roofline_sparse = {"kernel": "block_sparse_attn", "bound": "tensor", "achieved": round(sparse_tf, 2),
+                       "peak": peak_sus, "unit": "TFLOP/s", "frac": round(sparse_tf / peak_sus, 4)}
+    hbm = peaks.get("hbm_gbs")
+    perm_bytes = 2 * wl.heads * wl.N * wl.d * 2      # read + write of one tensor
+    perm_per_launch_ms = statistics.mean(perm_ms) / 4.0  # 4 permute launches per call
+    roofline_permute = {"kernel": "tile_major_permute", "bound": "hbm",
+                        "achieved": round(perm_bytes / (perm_per_launch_ms * 1e-3) / 1e9, 1),
+                        "peak": hbm, "unit": "GB/s",
+                        "frac": round(perm_bytes / (perm_per_launch_ms * 1e-3) / 1e9 / hbm, 4)}
+    mask_total = statistics.mean(mask_ms) + statistics.mean(radius_ms)
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Fourier-feature Q/K of grid position + noise, v ~ N(0,1))",
+        "config": {"workload": wl.name, "grid": [wl.F, wl.H, wl.W], "N": wl.N, "heads": wl.heads,
+                   "head_dim": wl.d, "block": [wl.block_q, wl.block_k], "tile": list(wl.tile),
+                   "gamma": wl.gamma, "vote": wl.vote, "tau": round(pipe.tau, 6),
+                   "kept_fraction": round(kept, 4), "sparse_calls_per_warmup": calls,
+                   "l2": "inputs larger than L2 (774 MB per tensor)", "parallelism": f"independent x{world}"},
+        "sparse_ms_per_call": round(s_ms, 3), "sparse_tflops_kept": round(sparse_tf, 2),
+        "dense_ms_per_call": round(d_ms, 3), "dense_tflops": round(dense_tf, 2),
+        "mask_ms": round(statistics.mean(mask_ms), 3), "radius_ms": round(statistics.mean(radius_ms), 4),
+        "permute_ms_per_call": round(statistics.mean(perm_ms), 3),
+        "overhead_vs_sparse": {"mask_plus_radius_ms": round(mask_total, 3),
+                               "ratio_to_4_sparse_calls": round(mask_total / (calls * s_ms), 4)},
+        "roofline": roofline, "roofline_sparse": roofline_sparse, "roofline_permute": roofline_permute,
+        "clocks": clocks, "gpu_launches": launches,
+    }
+
+    # ---- end to end: host (pinned) inputs copied in, O copied back, every call
+    e2e = e2e_run(pipe, host, dev, calls, args, device, world)
+    out["e2e"] = {"value": round(world * fl_step / (e2e["ms"] * 1e-3) / 1e12, 3), "unit": UNIT,
+                  "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                  "ms_per_step": round(e2e["ms"], 3)}
+    if rank == 0 and world == 1:
+        out["cpu_baseline"] = cpu_baseline(args, Q, K, V, pipe, kept_pairs, fl_step)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def e2e_run(pipe, host, dev, calls, args, device, world):
+    import torch.distributed as dist
+    out_host = torch.empty(pipe.O.shape, dtype=pipe.O.dtype).pin_memory()
+    h2d = d2h = 0
+
+    def step():
+        nonlocal h2d, d2h
+        # warm-up call: Q, K, V in
+        for i in range(3):
+            dev[i].copy_(host[i], non_blocking=True)
+            h2d += host[i].numel() * host[i].element_size()
+        pipe.warmup_call(dev[0], dev[1], dev[2], None)
+        out_host.copy_(pipe.O, non_blocking=True)
+        d2h += out_host.numel() * out_host.element_size()
+        for c in range(calls):
+            q, k = dev[3 + 2 * c], dev[4 + 2 * c]
+            for hsrc, d_ in ((host[3 + 2 * c], q), (host[4 + 2 * c], k), (host[2], dev[2])):
+                d_.copy_(hsrc, non_blocking=True)
+                h2d += hsrc.numel() * hsrc.element_size()
+            pipe.sparse_call(q, k, dev[2], None)
+            out_host.copy_(pipe.O, non_blocking=True)
+            d2h += out_host.numel() * out_host.element_size()
+
+    for _ in range(min(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    h2d = d2h = 0
+    if world > 1:
+        dist.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(1, min(args.steps, 3))
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"ms": ms / steps, "h2d": h2d // steps, "d2h": d2h // steps}
+
+
+# ------------------------------------------------------------- CPU baselines
+
+def oracle_throughput(Q, K, V, wl, tau, kept_frac, budget_s=15.0):
+    """The oracle (as it stands) on a bounded sample of one step's work: dense
+    attention + entropy rows, radius for all queries of one head, brute-force
+    mask rows, sparse attention rows.  Returns the extrapolated step time (s)
+    and what was sampled."""
+    from oracle import tra_oracle as O
+    N, d = wl.N, wl.d
+    scale = 1.0 / math.sqrt(d)
+    grid = (wl.F, wl.H, wl.W)
+    pi = O.tile_major_order(*grid, wl.tile)
+    c = O.token_coords(*grid)[pi]
+    q = O.permute(Q[0:1].double().numpy(), pi)[0]
+    k = O.permute(K[0:1].double().numpy(), pi)[0]
+    v = O.permute(V[0:1].double().numpy(), pi)[0]
+    rows = np.arange(0, 256)
+    t0 = time.perf_counter()
+    _, Hs, _ = O.attention_rows(q, k, v, scale, rows)
+    t_dense_row = (time.perf_counter() - t0) / len(rows)
+    # radius of every query of one head (entropy stand-in: the sampled values tiled)
+    Hfull = np.resize(Hs, N)
+    t0 = time.perf_counter()
+    r = O.radius(Hfull, c[:, 2], tau, wl.gamma, wl.F, N).astype(np.float32)
+    t_radius_head = time.perf_counter() - t0
+    phi32 = O.phi(np.arange(wl.F), wl.gamma).astype(np.float32)
+    t0 = time.perf_counter()
+    bm = O.block_mask(r, phi32, c, wl.block_q, wl.block_k, wl.vote, qblocks=[0, 1])
+    t_mask_row = (time.perf_counter() - t0) / 2
+    nkb = wl.nkb
+    mrow = np.zeros((wl.nqb, nkb), bool)
+    mrow[0] = bm[0]
+    mrow[1] = bm[1]
+    t0 = time.perf_counter()
+    O.sparse_attention_rows(q, k, v, mrow, wl.block_q, wl.block_k, scale, np.arange(0, 256))
+    t_sparse_row_measured = (time.perf_counter() - t0) / 256
+    # the oracle's sparse row costs like a dense row over the kept keys; scale the
+    # measured row (kept fraction of its own rows) to the workload's kept fraction
+    own = max(1e-9, float(bm.mean()))
+    t_sparse_row = t_sparse_row_measured * kept_frac / own if own > 0 else t_sparse_row_measured
+    heads = wl.heads
+    t_step = (heads * N * t_dense_row + heads * t_radius_head + heads * wl.nqb * t_mask_row
+              + wl.sparse_calls * heads * N * t_sparse_row)
+    sample = ("one head: 256 dense+entropy rows, radius of all 75600 queries, 2 brute-force mask "
+              "block rows, 256 sparse rows; extrapolated to 40 heads x (1 dense + 4 sparse calls)")
+    return t_step, sample
+
+
+def host_threads():
+    """Threads the oracle's numpy/BLAS calls actually use."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(args, Q, K, V, pipe, kept_pairs, fl_step):
+    wl = WL
+    kept_frac = kept_pairs / (wl.heads * wl.N * wl.N)
+    t_step, sample = oracle_throughput(Q, K, V, wl, pipe.tau, kept_frac)
+    return {"value": round(fl_step / t_step / 1e12, 6), "unit": UNIT,
+            "cores": host_threads(), "kind": "oracle", "sample": sample,
+            "extrapolated_step_s": round(t_step, 1)}
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return
+    wl = WL
+    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, 1, wl.d, wl.seed, wl.q_scale, "bf16")
+    kept = wl.kept_target
+    fl_sparse = 4.0 * wl.d * wl.N * wl.N * wl.heads * kept
+    fl_step = 4.0 * wl.d * wl.N * wl.N * wl.heads + wl.sparse_calls * fl_sparse
+    times = []
+    sample = ""
+    for i in range(args.warmup + args.steps):
+        t_step, sample = oracle_throughput(Q, K, V, wl, 0.01, kept)
+        if i >= args.warmup:
+            times.append(t_step)
+    t = statistics.mean(times)
+    v = fl_step / t / 1e12
+    out = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": UNIT,
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(t * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": wl.name, "kept_fraction": kept},
+           "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": host_threads(),
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def kernel_case(args):
+    """Small single-kernel cases for profiler captures (inputs > L2, < 1 GB):
+    dense / sparse: 40 heads x 16384 tokens x d=128 bf16 (168 MB per tensor);
+    mask: the 21x45x80 grid, 40 heads, radii from entropies near ln N;
+    permute: one 21x45x80 x 40-head x 128 bf16 tensor.  Runs the kernel
+    `--reps` times and prints the mean CUDA-event time per launch."""
+    from entropy_adaptive_radius_b200 import tra
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev).manual_seed(0)
+    heads, N, d = 40, 16384, 128
+    reps = args.reps
+    if args.case in ("dense", "sparse"):
+        Q = (torch.randn(heads, N, d, generator=g, device=dev) * 2).to(torch.bfloat16)
+        K = torch.randn(heads, N, d, generator=g, device=dev).to(torch.bfloat16)
+        V = torch.randn(heads, N, d, generator=g, device=dev).to(torch.bfloat16)
+        O_ = torch.empty_like(Q)
+        H = torch.empty(heads, N, dtype=torch.float32, device=dev)
+        nb = N // 128
+        mask = inputs.synthetic_block_mask(heads, nb, nb, seed=0, density=0.12)
+        rp, ci = inputs.csr_from_block_mask(mask)
+        rpd, cid = torch.from_numpy(rp.ravel()).to(dev), torch.from_numpy(ci).to(dev)
+        kept = int(mask.sum()) * 128 * 128
+        if args.case == "dense":
+            fn = lambda: tra.tra_dense_attn_entropy(Q, K, V, O_, H)  # noqa: E731
+            flops = 4.0 * d * N * N * heads
+        else:
+            fn = lambda: tra.tra_block_sparse_attn(Q, K, V, O_, rpd, cid, 128, 128)  # noqa: E731
+            flops = 4.0 * d * kept
+        unit = ("TFLOP/s", flops / 1e12)
+    elif args.case == "mask":
+        wl = WL
+        grid = (wl.F, wl.H, wl.W)
+        Hs = inputs.synthetic_entropy(wl.heads, wl.N, 0, math.log(wl.N) - 2.0, math.log(wl.N))
+        Hd = torch.from_numpy(Hs).to(dev)
+        r = torch.empty_like(Hd)
+        phi = torch.empty(wl.F, dtype=torch.float32, device=dev)
+        tra.tra_budget_radius(Hd, r, grid, 0.05, wl.gamma, wl.tile, phi_out=phi)
+        ws = tra.workspace_tensor(tra.tra_mask_workspace_size(wl.heads, grid, 128, 128, wl.tile), dev)
+        rp = torch.empty(wl.heads * (wl.nqb + 1), dtype=torch.int32, device=dev)
+        ci = torch.empty(wl.heads * wl.nqb * wl.nkb, dtype=torch.int32, device=dev)
+        nnz = torch.empty(1, dtype=torch.int32, device=dev)
+        fn = lambda: tra.tra_build_block_mask(r, phi, grid, 128, 128, 1, rp, ci, nnz, ws, wl.tile)  # noqa: E731
+        unit = ("Gpairs/s", wl.heads * wl.N * wl.N / 1e9)
+    else:
+        wl = WL
+        grid = (wl.F, wl.H, wl.W)
+        X = torch.randn(wl.heads, wl.N, wl.d, generator=g, device=dev).to(torch.bfloat16)
+        Y = torch.empty_like(X)
+        fn = lambda: tra.tra_tile_major_permute(X, Y, grid, wl.tile)  # noqa: E731
+        unit = ("GB/s", 2 * X.numel() * 2 / 1e9)
+    fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    if tra.tra_get_device_error() != 0:
+        raise RuntimeError("device-side wait timed out")
+    ms = s.elapsed_time(e) / reps
+    print(json.dumps({"case": args.case, "ms_per_launch": round(ms, 4),
+                      "rate": round(unit[1] / (ms * 1e-3), 2), "unit": unit[0]}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=["dense", "sparse", "mask", "permute"], default=None,
+                    help="run one kernel on a small case (for profiler captures)")
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="tra", choices=["tra", "reference"])
+    args = ap.parse_args()
+    rank, world, local = dist_env()
+    if args.case is not None:
+        kernel_case(args)
+        return
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    gpu_arm(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

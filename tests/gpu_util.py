@@ -38,7 +38,8 @@ def check_close(x_gpu, x_ref, tol, what=""):
     a = to64(x_gpu) if isinstance(x_gpu, torch.Tensor) else np.asarray(x_gpu, np.float64)
     b = np.asarray(x_ref, np.float64)
     both_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
-    err = np.where(both_inf, 0.0, np.abs(a - b))
+    with np.errstate(invalid="ignore"):
+        err = np.where(both_inf, 0.0, np.abs(a - b))
     mx = float(np.nanmax(err)) if err.size else 0.0
     assert not np.isnan(err).any(), f"{what}: NaN mismatch"
     assert mx <= tol, f"{what}: max abs err {mx:.3e} > {tol}"

@@ -97,11 +97,13 @@ def test_budget_radius(wl, tau):
     r = torch.empty_like(Hd)
     phi = torch.empty(wl.F, dtype=torch.float32, device="cuda")
     tra.tra_budget_radius(Hd, r, (wl.F, wl.H, wl.W), tau, wl.gamma, wl.tile, phi_out=phi)
-    phi_ref = O.phi(np.arange(wl.F), wl.gamma)
+    # the C ABI takes tau and gamma as float32: the oracle gets those same values
+    tau32, gamma32 = float(np.float32(tau)), float(np.float32(wl.gamma))
+    phi_ref = O.phi(np.arange(wl.F), gamma32)
     np.testing.assert_allclose(phi.cpu().numpy(), phi_ref, rtol=1e-7, atol=0)
     rg = r.cpu().numpy().astype(np.float64)
     for h in range(heads):
-        ref = O.radius(Hs[h].astype(np.float64), t_tm, tau, wl.gamma, wl.F, N)
+        ref = O.radius(Hs[h].astype(np.float64), t_tm, tau32, gamma32, wl.F, N)
         fin = np.isfinite(ref)
         np.testing.assert_allclose(rg[h][fin], ref[fin], rtol=2e-6, atol=0)
         assert np.array_equal(np.isinf(rg[h]), np.isinf(ref))
