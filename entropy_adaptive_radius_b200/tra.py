@@ -52,6 +52,8 @@ _PROTOS = {
     "tra_mask_workspace_size": (_c_size, [_c_int, Grid, Tile, _c_int, _c_int]),
     "tra_build_block_mask": (_c_int, [_vp, _vp, _c_int, Grid, Tile, _c_int, _c_int, _c_int, _vp,
                                       _vp, _c_ll, _vp, _vp, _c_size, _vp]),
+    "tra_build_block_mask_noalloc": (_c_int, [_vp, _vp, _c_int, Grid, Tile, _c_int, _c_int, _c_int,
+                                              _vp, _vp, _c_ll, _vp, _vp]),
     "tra_block_sparse_attn": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                                        _c_int, _c_int, _c_float, _vp]),
     "tra_get_device_error": (_c_int, [ctypes.POINTER(_c_int), _vp]),
@@ -171,6 +173,23 @@ def tra_build_block_mask(r, phi, grid, block_q, block_k, vote, row_ptr, col_idx,
         _p(col_idx), col_idx.numel(), _p(nnz), _p(workspace), workspace.numel(),
         _stream(stream)))
     return row_ptr, col_idx, nnz
+
+
+def tra_build_block_mask_noalloc(r, phi, grid, block_q, block_k, vote, row_ptr, col_idx, nnz,
+                                 tile=(1, 4, 4), stream=None):
+    """Same CSR as tra_build_block_mask, for callers that cannot pass scratch
+    memory: the library uses its built-in buffer of TRA_MASK_STATIC_SCRATCH_BYTES
+    (8 MiB per device).  Calls that overlap on the GPU share that buffer and
+    race; issue them in order on one stream."""
+    _contig(r, phi, row_ptr, col_idx, nnz)
+    heads = r.shape[0]
+    _check("tra_build_block_mask_noalloc", lib().tra_build_block_mask_noalloc(
+        _p(r), _p(phi), heads, _grid(grid), _tile(tile), block_q, block_k, vote, _p(row_ptr),
+        _p(col_idx), col_idx.numel(), _p(nnz), _stream(stream)))
+    return row_ptr, col_idx, nnz
+
+
+MASK_STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 
 def tra_block_sparse_attn(Q, K, V, O, row_ptr, col_idx, block_q, block_k, lse=None, scale=None,

@@ -175,6 +175,39 @@ tra_status tra_build_block_mask(const float* r, const float* phi, int heads, tra
                                 void* workspace, size_t workspace_bytes, tra_stream_t stream);
 
 /*
+ * Size in bytes of the scratch buffer built into the library for
+ * tra_build_block_mask_noalloc.  Every GPU that loads the library holds this
+ * much device memory until the process exits.
+ */
+#define TRA_MASK_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+/*
+ * tra_build_block_mask for callers that cannot allocate or pass scratch
+ * memory, such as a plugin that receives only its input and output tensors
+ * from a host framework that owns all device memory, or a latency-critical
+ * caller that must not allocate mid-run.  The pages have no counterpart for
+ * this call: it is a packaging variant of the fused mask above.
+ *
+ * Inputs, outputs, rules and results are those of tra_build_block_mask; only
+ * workspace / workspace_bytes are gone.  Scratch comes from one buffer of
+ * TRA_MASK_STATIC_SCRATCH_BYTES compiled into the library (one per device).
+ * A problem that needs more (tra_mask_workspace_size(...) larger than that) is
+ * refused with TRA_ERR_WORKSPACE before anything is launched.  The call
+ * allocates nothing and calls no allocator.
+ *
+ * The first call on each device looks up the device address of the built-in
+ * buffer (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  All calls on a device share the buffer and
+ * leave their data in it: calls whose kernels overlap on the GPU (different
+ * streams or host threads) race and corrupt each other's results, so issue
+ * them in order on one stream.
+ */
+tra_status tra_build_block_mask_noalloc(const float* r, const float* phi, int heads,
+                                        tra_grid grid, tra_tile tile, int block_q, int block_k,
+                                        int vote_threshold, int* row_ptr, int* col_idx,
+                                        long long col_capacity, int* nnz, tra_stream_t stream);
+
+/*
  * Block-sparse attention over the kept blocks (§2 "TRA pipeline": the
  * block-sparse mask drives a block-sparse attention backend; reuse across
  * sparse steps).  Exact softmax over every token of the kept key blocks of
