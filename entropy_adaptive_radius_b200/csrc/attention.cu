@@ -107,6 +107,34 @@ __device__ __forceinline__ void tmem_st16f(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// 2^x on the MUFU unit (flushes subnormal results to zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
+        "=f"(v[7]), "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]),
+        "=f"(v[14]), "=f"(v[15]), "=f"(v[16]), "=f"(v[17]), "=f"(v[18]), "=f"(v[19]),
+        "=f"(v[20]), "=f"(v[21]), "=f"(v[22]), "=f"(v[23]), "=f"(v[24]), "=f"(v[25]),
+        "=f"(v[26]), "=f"(v[27]), "=f"(v[28]), "=f"(v[29]), "=f"(v[30]), "=f"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+
 template <int N>
 __device__ __forceinline__ void freg_fence(float* v) {
 #pragma unroll
@@ -371,8 +399,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
+      if constexpr (BK % 32 == 0) {
 #pragma unroll
-      for (int c = 0; c < BK / 16; ++c) tmem_ld16f(tmem + tl + b * BK + c * 16, sv + c * 16);
+        for (int c = 0; c < BK / 32; ++c) tmem_ld32f(tmem + tl + b * BK + c * 32, sv + c * 32);
+      } else {
+#pragma unroll
+        for (int c = 0; c < BK / 16; ++c) tmem_ld16f(tmem + tl + b * BK + c * 16, sv + c * 16);
+      }
       tmem_wait_ld();
       freg_fence<BK>(sv);
       tc_fence_before();
@@ -383,37 +416,93 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kb < 0 || kb >= p.nkb) nvalid = 0;
         else if (p.G > 1 && !((qbmap[g * 32 + (kb >> 5)] >> (kb & 31)) & 1u)) nvalid = 0;
       }
-      float bmax = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BK; ++c) {
-        const float u = c < nvalid ? sv[c] * p.scale_log2 : -INFINITY;
-        sv[c] = u;
-        bmax = fmaxf(bmax, u);
-      }
-      const float m_new = fmaxf(m_ref, bmax);
+      // Running max with lazy rescale: the reference m_ref moves only when the
+      // block max exceeds it by more than 2^8; then Z, A (and O, below) are
+      // scaled by alpha = 2^(m_ref - m_new).
       float alpha = 1.f;
       bool o_rescale = false;
-      if (m_new > m_ref + kRescaleLog2) {
-        if (m_ref != -INFINITY) {
-          alpha = exp2f(m_ref - m_new);
-          A = alpha * (A + (m_ref - m_new) * Z);
-          Z *= alpha;
-          o_rescale = j > 0;
+      auto update_max = [&](float bmax) {
+        const float m_new = fmaxf(m_ref, bmax);
+        if (m_new > m_ref + kRescaleLog2) {
+          if (m_ref != -INFINITY) {
+            alpha = ex2_approx(m_ref - m_new);
+            A = alpha * (A + (m_ref - m_new) * Z);
+            Z *= alpha;
+            o_rescale = j > 0;
+          }
+          m_ref = m_new;
         }
-        m_ref = m_new;
-      }
-      const float mc = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float zs = 0.f, as = 0.f;
+      };
+      uint32_t pk[BK / 2];  // P_j as packed bf16 pairs
+      if (__all_sync(0xffffffffu, nvalid >= BK)) {
+        // Unmasked block (every row of the warp sees all BK keys).
+        // Row max of the raw scores (scale > 0 commutes with max): four
+        // independent chains of 3-input max.
+        float mx[4];
 #pragma unroll
-      for (int c = 0; c < BK; ++c) {
-        const float x = sv[c] - mc;
-        const float pr = exp2f(x);
-        zs += pr;
-        if constexpr (DENSE) as += pr > 0.f ? pr * x : 0.f;
-        sv[c] = pr;
+        for (int i = 0; i < 4; ++i) mx[i] = fmaxf(sv[i], sv[4 + i]);
+#pragma unroll
+        for (int c = 8; c < BK; c += 8) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) mx[i] = fmax3(mx[i], sv[c + i], sv[c + 4 + i]);
+        }
+        update_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2);
+        // m_ref is finite here.  x = s * scale * log2(e) - m_ref, p = 2^x,
+        // Z += p, A += p * x, two lanes per instruction, four partial sums.
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(-m_ref, -m_ref);
+        float2 z2[4], a2[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) z2[i] = a2[i] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < BK / 2; ++c) {
+          const float2 x = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nm2);
+          const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          z2[c & 3] = __fadd2_rn(z2[c & 3], pr);
+          if constexpr (DENSE) a2[c & 3] = __ffma2_rn(pr, x, a2[c & 3]);
+          pk[c] = pack_bf16(pr.x, pr.y);
+        }
+        const float2 zz = __fadd2_rn(__fadd2_rn(z2[0], z2[1]), __fadd2_rn(z2[2], z2[3]));
+        Z += zz.x + zz.y;
+        if constexpr (DENSE) {
+          const float2 aa = __fadd2_rn(__fadd2_rn(a2[0], a2[1]), __fadd2_rn(a2[2], a2[3]));
+          A += aa.x + aa.y;
+        }
+      } else if (__all_sync(0xffffffffu, nvalid <= 0)) {
+        // No row of the warp keeps this block: P = 0, statistics unchanged.
+#pragma unroll
+        for (int c = 0; c < BK / 2; ++c) pk[c] = 0u;
+      } else {
+        // Partly masked block (the last, partial key block, or rows of a
+        // merged list that do not keep this block): masked keys get -inf.
+        float bm0 = -INFINITY, bm1 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BK; c += 2) {
+          const float u0 = c < nvalid ? sv[c] * p.scale_log2 : -INFINITY;
+          const float u1 = c + 1 < nvalid ? sv[c + 1] * p.scale_log2 : -INFINITY;
+          sv[c] = u0;
+          sv[c + 1] = u1;
+          bm0 = fmaxf(bm0, u0);
+          bm1 = fmaxf(bm1, u1);
+        }
+        update_max(fmaxf(bm0, bm1));
+        const float mc = (m_ref == -INFINITY) ? 0.f : m_ref;
+        float zs0 = 0.f, zs1 = 0.f, as0 = 0.f, as1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < BK / 2; ++c) {
+          const float x0 = sv[2 * c] - mc, x1 = sv[2 * c + 1] - mc;
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          zs0 += p0;
+          zs1 += p1;
+          if constexpr (DENSE) {
+            as0 += p0 > 0.f ? p0 * x0 : 0.f;
+            as1 += p1 > 0.f ? p1 * x1 : 0.f;
+          }
+          pk[c] = pack_bf16(p0, p1);
+        }
+        Z += zs0 + zs1;
+        A += as0 + as1;
       }
-      Z += zs;
-      A += as;
 
       if (j > 0) {
         ok = mbar_wait(pv_done, (j - 1) & 1, abort, p.err, kErrWaitPVDone);
@@ -438,10 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c8 = 0; c8 < BK / 8; ++c8) {
         const uint32_t addr = sP + (c8 >> 3) * (BM * 128) + row * 128 + (((c8 & 7) ^ (row & 7)) << 4);
-        st_shared_v4(addr, pack_bf16(sv[c8 * 8 + 0], sv[c8 * 8 + 1]),
-                     pack_bf16(sv[c8 * 8 + 2], sv[c8 * 8 + 3]),
-                     pack_bf16(sv[c8 * 8 + 4], sv[c8 * 8 + 5]),
-                     pack_bf16(sv[c8 * 8 + 6], sv[c8 * 8 + 7]));
+        st_shared_v4(addr, pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
