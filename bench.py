@@ -151,11 +151,12 @@ class Pipeline:
             tra.tra_mask_workspace_size(h, self.grid, wl.block_q, wl.block_k, wl.tile), device)
         self.launches = 0
         self.tau = 1.0
+        self.vote = wl.vote
 
     def mask(self, tau):
         w, t = self.wl, self.tra
         t.tra_budget_radius(self.H, self.r, self.grid, tau, w.gamma, w.tile, phi_out=self.phi)
-        t.tra_build_block_mask(self.r, self.phi, self.grid, w.block_q, w.block_k, w.vote,
+        t.tra_build_block_mask(self.r, self.phi, self.grid, w.block_q, w.block_k, self.vote,
                                self.row_ptr, self.col_idx, self.nnz, self.ws, w.tile)
         self.launches += 5
 
@@ -172,7 +173,7 @@ class Pipeline:
                             phi_out=self.phi)
         e[3].record()
         t.tra_build_block_mask(self.r, self.phi, self.grid, self.wl.block_q, self.wl.block_k,
-                               self.wl.vote, self.row_ptr, self.col_idx, self.nnz, self.ws,
+                               self.vote, self.row_ptr, self.col_idx, self.nnz, self.ws,
                                self.wl.tile)
         e[4].record()
         t.tra_inverse_permute(self.Otm, self.O, self.grid, self.wl.tile)
@@ -199,6 +200,50 @@ class Pipeline:
 
     def kept_fraction(self):
         return int(self.nnz.item()) / (self.wl.heads * self.nqb * self.nkb)
+
+
+WORKLOADS = {"wan14b": workloads.WAN14B, "wan13b": workloads.WAN13B,
+             "hunyuan": workloads.HUNYUAN, "tiny": workloads.TINY}
+
+
+def l2_note(wl):
+    mb = wl.heads * wl.N * wl.d * 2 / 1e6
+    if mb > 126:
+        return f"inputs larger than L2 ({mb:.0f} MB per tensor)"
+    return f"inputs fit in L2 ({mb:.1f} MB per tensor); L2 not flushed"
+
+
+def full_csr(heads, N, block, device):
+    """CSR that keeps every (query block, key block) pair."""
+    nqb = nkb = -(-N // block)
+    idx = torch.arange(heads * (nqb + 1), dtype=torch.int64)
+    rp = (idx // (nqb + 1) * nqb + idx % (nqb + 1)) * nkb
+    ci = torch.arange(nkb, dtype=torch.int32).repeat(heads * nqb)
+    return rp.to(torch.int32).to(device), ci.to(device)
+
+
+def time_ms(fn, reps=5):
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        torch.cuda.synchronize()
+        ts.append(s.elapsed_time(e))
+    return statistics.median(ts)
+
+
+def plain_dense_ms(pipe, wl, device, reps=3):
+    """Dense attention without entropy: the block-sparse kernel over a CSR
+    that keeps every 128 x 128 block (the dense call's own tiling), timed
+    outside the step."""
+    rp, ci = full_csr(wl.heads, wl.N, 128, device)
+    t = pipe.tra
+    return time_ms(lambda: t.tra_block_sparse_attn(pipe.Qtm, pipe.Ktm, pipe.Vtm, pipe.Otm, rp, ci,
+                                                   128, 128), reps)
 
 
 def calibrate_tau(pipe, target, log):
@@ -230,10 +275,10 @@ def gpu_arm(args, rank, world, local):
     if world > 1:
         dist.init_process_group("nccl", device_id=device,
                                 timeout=__import__("datetime").timedelta(seconds=600))
-    wl = WL
+    wl = WORKLOADS[args.workload]
     calls = wl.sparse_calls
     t0 = time.time()
-    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed, wl.q_scale, "bf16",
+    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed, wl.q_scale, wl.dtype,
                               head_offset=rank * wl.heads)
     pert = [(inputs.perturb(Q, wl.seed, c, 0, head_offset=rank * wl.heads),
              inputs.perturb(K, wl.seed, c, 1, head_offset=rank * wl.heads)) for c in range(1, calls + 1)]
@@ -248,7 +293,7 @@ def gpu_arm(args, rank, world, local):
     # dense warm-up once to get H, then calibrate tau on it
     pipe.warmup_call(Qd, Kd, Vd, None)
     torch.cuda.synchronize()
-    pipe.tau = calibrate_tau(pipe, wl.kept_target, log)
+    pipe.tau = calibrate_tau(pipe, wl.kept_target, log) if wl.kept_target else wl.tau
     pipe.warmup_call(Qd, Kd, Vd, None)
     torch.cuda.synchronize()
     kept = pipe.kept_fraction()
@@ -297,6 +342,10 @@ def gpu_arm(args, rank, world, local):
     if tra.tra_get_device_error() != 0:
         raise RuntimeError("device-side wait timed out in the timed region")
 
+    # plain dense attention (no entropy) for the entropy-overhead term: the
+    # sparse kernel over a CSR that keeps every block
+    plain_ms = plain_dense_ms(pipe, wl, device)
+
     # per-kernel times (launching stream = current stream)
     dense_ms, sparse_ms, mask_ms, radius_ms, perm_ms = [], [], [], [], []
     for kind, e in rec:
@@ -340,13 +389,18 @@ def gpu_arm(args, rank, world, local):
                    "head_dim": wl.d, "block": [wl.block_q, wl.block_k], "tile": list(wl.tile),
                    "gamma": wl.gamma, "vote": wl.vote, "tau": round(pipe.tau, 6),
                    "kept_fraction": round(kept, 4), "sparse_calls_per_warmup": calls,
-                   "l2": "inputs larger than L2 (774 MB per tensor)", "parallelism": f"independent x{world}"},
+                   "l2": l2_note(wl), "parallelism": f"independent x{world}"},
         "sparse_ms_per_call": round(s_ms, 3), "sparse_tflops_kept": round(sparse_tf, 2),
         "dense_ms_per_call": round(d_ms, 3), "dense_tflops": round(dense_tf, 2),
         "mask_ms": round(statistics.mean(mask_ms), 3), "radius_ms": round(statistics.mean(radius_ms), 4),
         "permute_ms_per_call": round(statistics.mean(perm_ms), 3),
-        "overhead_vs_sparse": {"mask_plus_radius_ms": round(mask_total, 3),
-                               "ratio_to_4_sparse_calls": round(mask_total / (calls * s_ms), 4)},
+        "overhead_vs_sparse": {
+            "entropy_ms": round(d_ms - plain_ms, 3), "plain_dense_ms": round(plain_ms, 3),
+            "mask_plus_radius_ms": round(mask_total, 3),
+            "total_ms": round(max(0.0, d_ms - plain_ms) + mask_total, 3),
+            "ratio_to_sparse_calls": round((max(0.0, d_ms - plain_ms) + mask_total) / (calls * s_ms), 4),
+            "unamortised_ratio_to_1_call": round((max(0.0, d_ms - plain_ms) + mask_total) / s_ms, 4),
+            "sparse_calls": calls},
         "roofline": roofline, "roofline_sparse": roofline_sparse, "roofline_permute": roofline_permute,
         "clocks": clocks, "gpu_launches": launches,
     }
@@ -357,7 +411,7 @@ def gpu_arm(args, rank, world, local):
                   "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                   "ms_per_step": round(e2e["ms"], 3)}
     if rank == 0 and world == 1:
-        out["cpu_baseline"] = cpu_baseline(args, Q, K, V, pipe, kept_pairs, fl_step)
+        out["cpu_baseline"] = cpu_baseline(args, Q, K, V, pipe, kept_pairs, fl_step, wl)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -425,7 +479,7 @@ def oracle_throughput(Q, K, V, wl, tau, kept_frac, budget_s=15.0):
     q = O.permute(Q[0:1].double().numpy(), pi)[0]
     k = O.permute(K[0:1].double().numpy(), pi)[0]
     v = O.permute(V[0:1].double().numpy(), pi)[0]
-    rows = np.arange(0, 256)
+    rows = np.arange(0, min(256, N))
     t0 = time.perf_counter()
     _, Hs, _ = O.attention_rows(q, k, v, scale, rows)
     t_dense_row = (time.perf_counter() - t0) / len(rows)
@@ -436,15 +490,15 @@ def oracle_throughput(Q, K, V, wl, tau, kept_frac, budget_s=15.0):
     t_radius_head = time.perf_counter() - t0
     phi32 = O.phi(np.arange(wl.F), wl.gamma).astype(np.float32)
     t0 = time.perf_counter()
-    bm = O.block_mask(r, phi32, c, wl.block_q, wl.block_k, wl.vote, qblocks=[0, 1])
+    bm = O.block_mask(r, phi32, c, wl.block_q, wl.block_k, wl.vote, qblocks=[0, min(1, wl.nqb - 1)])
     t_mask_row = (time.perf_counter() - t0) / 2
     nkb = wl.nkb
     mrow = np.zeros((wl.nqb, nkb), bool)
     mrow[0] = bm[0]
     mrow[1] = bm[1]
     t0 = time.perf_counter()
-    O.sparse_attention_rows(q, k, v, mrow, wl.block_q, wl.block_k, scale, np.arange(0, 256))
-    t_sparse_row_measured = (time.perf_counter() - t0) / 256
+    O.sparse_attention_rows(q, k, v, mrow, wl.block_q, wl.block_k, scale, rows)
+    t_sparse_row_measured = (time.perf_counter() - t0) / len(rows)
     # the oracle's sparse row costs like a dense row over the kept keys; scale the
     # measured row (kept fraction of its own rows) to the workload's kept fraction
     own = max(1e-9, float(bm.mean()))
@@ -452,8 +506,9 @@ def oracle_throughput(Q, K, V, wl, tau, kept_frac, budget_s=15.0):
     heads = wl.heads
     t_step = (heads * N * t_dense_row + heads * t_radius_head + heads * wl.nqb * t_mask_row
               + wl.sparse_calls * heads * N * t_sparse_row)
-    sample = ("one head: 256 dense+entropy rows, radius of all 75600 queries, 2 brute-force mask "
-              "block rows, 256 sparse rows; extrapolated to 40 heads x (1 dense + 4 sparse calls)")
+    sample = (f"one head: 256 dense+entropy rows, radius of all {N} queries, 2 brute-force mask "
+              f"block rows, 256 sparse rows; extrapolated to {heads} heads x (1 dense + "
+              f"{wl.sparse_calls} sparse calls)")
     return t_step, sample
 
 
@@ -469,8 +524,7 @@ def host_threads():
     return os.cpu_count() or 1
 
 
-def cpu_baseline(args, Q, K, V, pipe, kept_pairs, fl_step):
-    wl = WL
+def cpu_baseline(args, Q, K, V, pipe, kept_pairs, fl_step, wl):
     kept_frac = kept_pairs / (wl.heads * wl.N * wl.N)
     t_step, sample = oracle_throughput(Q, K, V, wl, pipe.tau, kept_frac)
     return {"value": round(fl_step / t_step / 1e12, 6), "unit": UNIT,
@@ -478,12 +532,64 @@ def cpu_baseline(args, Q, K, V, pipe, kept_pairs, fl_step):
             "extrapolated_step_s": round(t_step, 1)}
 
 
+def sweep_arm(args):
+    """Density sweep at the 21x45x80, 40-head shape: for each vote threshold
+    and target kept fraction, tau is bisected to the target (or the nearest
+    reachable fraction: every query keeps its own position in every frame, so
+    the fraction has a floor), then the block-sparse call is timed against the
+    dense calls.  One JSON line per point."""
+    from entropy_adaptive_radius_b200 import tra
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    wl = workloads.SWEEP
+    log = lambda m: print(f"[sweep] {m}", file=sys.stderr, flush=True)  # noqa: E731
+    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed, wl.q_scale, wl.dtype)
+    Qd, Kd, Vd = Q.to(device), K.to(device), V.to(device)
+    pipe = Pipeline(wl, device)
+    pipe.warmup_call(Qd, Kd, Vd, None)
+    torch.cuda.synchronize()
+    dense_ms = time_ms(lambda: tra.tra_dense_attn_entropy(pipe.Qtm, pipe.Ktm, pipe.Vtm, pipe.Otm,
+                                                         pipe.H), 3)
+    plain_ms = plain_dense_ms(pipe, wl, device)
+    peaks, kind = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    for vote in wl.sweep_votes:
+        pipe.vote = vote
+        pipe.mask(1e-12)
+        floor = pipe.kept_fraction()
+        for target in wl.sweep:
+            if target >= 1.0:
+                ms, kept, tau, pairs = plain_ms, 1.0, None, wl.heads * wl.N * wl.N
+            else:
+                tau = calibrate_tau(pipe, target, log)
+                pipe.mask(tau)
+                kept = pipe.kept_fraction()
+                rp = pipe.row_ptr.cpu().numpy()
+                ci = pipe.col_idx[: int(pipe.nnz.item())].cpu().numpy()
+                pairs = kept_pair_tokens(rp, ci, wl.heads, wl.N, wl.block_q, wl.block_k)
+                ms = time_ms(lambda: tra.tra_block_sparse_attn(
+                    pipe.Qtm, pipe.Ktm, pipe.Vtm, pipe.Otm, pipe.row_ptr, pipe.col_idx,
+                    wl.block_q, wl.block_k), 5)
+                mask_ms = time_ms(lambda: pipe.mask(tau), 3)
+            tf = 4.0 * wl.d * pairs / (ms * 1e-3) / 1e12
+            row = {"workload": wl.name, "vote": vote, "target_kept": target,
+                   "kept_fraction": round(kept, 4), "kept_floor": round(floor, 4),
+                   "tau": None if tau is None else round(tau, 8), "sparse_ms": round(ms, 3),
+                   "sparse_tflops_kept": round(tf, 1), "roofline_frac": round(tf / peak, 4),
+                   "peak": f"{peak} TFLOP/s ({kind} bf16 sustained)",
+                   "dense_entropy_ms": round(dense_ms, 3), "plain_dense_ms": round(plain_ms, 3),
+                   "speedup_vs_dense": round(dense_ms / ms, 3)}
+            if target < 1.0:
+                row["mask_ms"] = round(mask_ms, 3)
+            print(json.dumps(row), flush=True)
+
+
 def reference_arm(args, rank, world):
     if rank != 0:
         return
-    wl = WL
-    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, 1, wl.d, wl.seed, wl.q_scale, "bf16")
-    kept = wl.kept_target
+    wl = WORKLOADS.get(args.workload, WL)
+    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, 1, wl.d, wl.seed, wl.q_scale, wl.dtype)
+    kept = wl.kept_target if wl.kept_target else 1.0
     fl_sparse = 4.0 * wl.d * wl.N * wl.N * wl.heads * kept
     fl_step = 4.0 * wl.d * wl.N * wl.N * wl.heads + wl.sparse_calls * fl_sparse
     times = []
@@ -577,6 +683,9 @@ def main():
     ap.add_argument("--case", choices=["dense", "sparse", "mask", "permute"], default=None,
                     help="run one kernel on a small case (for profiler captures)")
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--workload", default="wan14b", choices=sorted(WORKLOADS) + ["sweep"],
+                    help="wan14b (default, the headline step), wan13b, hunyuan, tiny, or the "
+                         "density sweep")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
@@ -588,6 +697,9 @@ def main():
         return
     if args.impl == "reference":
         reference_arm(args, rank, world)
+        return
+    if args.workload == "sweep":
+        sweep_arm(args)
         return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -121,6 +121,27 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
+// 2^x for two lanes on the FMA pipe (Cody-Waite style reduction): x = n + f
+// with n = rint(x) (adding 1.5 * 2^23 leaves rint(x) in the low mantissa bits
+// of t), f in [-1/2, 1/2], 2^f from a degree-3 polynomial minimax in relative
+// error on that interval (max relative error 7.5e-5; coefficients fitted by
+// Remez exchange, see fit_exp2_poly.py), and 2^n applied by adding n to the
+// exponent field: bits(t) << 23 == n << 23 (mod 2^32).  x is clamped below at
+// -125 so the exponent stays in range; results there are below 2^-124.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(f, make_float2(0.055171669f, 0.055171669f),
+                        make_float2(0.24261112f, 0.24261112f));
+  q = __ffma2_rn(q, f, make_float2(0.69326099f, 0.69326099f));
+  q = __ffma2_rn(q, f, make_float2(0.99992807f, 0.99992807f));
+  return make_float2(__int_as_float((__float_as_int(t.x) << 23) + __float_as_int(q.x)),
+                     __int_as_float((__float_as_int(t.y) << 23) + __float_as_int(q.y)));
+}
+
 __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float* v) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -579,6 +600,492 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Two-warpgroup variant for 128-row query blocks and 128-key blocks.
+//
+// The CTA owns one 128-row query tile.  Its key-block list is split between
+// two softmax warpgroups: warpgroup w (warps 4w .. 4w+3) takes blocks
+// j = w, w + 2, w + 4, ... with its own TMEM score tile S_w, its own TMEM output
+// accumulator O_w, its own bf16 P_w buffer in shared memory and its own
+// running statistics (m_w, Z_w, A_w).  Each warpgroup therefore has two block
+// periods of tensor-core work to hide one softmax iteration, and each
+// scheduler has two softmax warps to issue from.  The MMA warp issues QK^T two
+// blocks ahead of PV (S_{j+2} as soon as warpgroup j mod 2 has read S_j), so a
+// score tile is ready when its warpgroup finishes the previous one.  K and V
+// have separate producer warps so that prefetching K never waits behind a V
+// slot that is still in use.  At the end the two partial results are merged
+// exactly:
+//   m = max(m_0, m_1),  a_w = 2^(m_w - m),  Z = a_0 Z_0 + a_1 Z_1,
+//   A = sum_w a_w (A_w + (m_w - m) Z_w),      O = (a_0 O_0 + a_1 O_1) / Z.
+// Warps: 0..7 softmax, 8 Q/K producer (and tensor-memory allocation), 9 MMA,
+// 10 V producer.
+// ---------------------------------------------------------------------------
+
+constexpr int kDualThreads = 352;  // 11 warps
+constexpr int kDualKWarp = 8;
+constexpr int kDualMmaWarp = 9;
+constexpr int kDualVWarp = 10;
+
+template <int D>
+struct DualCfg {
+  static constexpr int BK = 128;
+  static constexpr int NS = 2;
+  static constexpr int KCH = D / 64;
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BK * D * 2;
+  static constexpr int P_BYTES = 2 * BM * 128;  // one P_w buffer (128 rows x 128 keys bf16)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + NS * KV_BYTES;  // P_0, P_1
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int NUM_BARS = 1 + 4 * NS + 8 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + 256;
+  static constexpr int USED = OFF_MISC + 64;
+  static constexpr int SMEM = (USED < 120 * 1024 ? 120 * 1024 : USED) + 1024;
+  static constexpr int TMEM_COLS = 512;  // S_0, S_1 (128 each), O_0, O_1 (D each)
+  static_assert(2 * BK + 2 * D <= TMEM_COLS, "tensor memory");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(NUM_BARS * 8 <= 256, "barrier area");
+};
+
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <int D, bool DENSE>
+__global__ void __launch_bounds__(kDualThreads, 1)
+    attn_dual_kernel(const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using C = DualCfg<D>;
+  constexpr int NS = C::NS;
+  constexpr int BK = C::BK;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::OFF_Q;
+  const uint32_t sK = sbase + C::OFF_K;
+  const uint32_t sV = sbase + C::OFF_V;
+  const uint32_t sP = sbase + C::OFF_P;
+  const uint32_t bars = sbase + C::OFF_BAR;
+  const uint32_t bar_q = bars;
+  auto k_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto k_empty = [&](int s) { return bars + 8u * (1 + NS + s); };
+  auto v_full = [&](int s) { return bars + 8u * (1 + 2 * NS + s); };
+  auto v_empty = [&](int s) { return bars + 8u * (1 + 3 * NS + s); };
+  auto s_full = [&](int w) { return bars + 8u * (1 + 4 * NS + w); };
+  auto s_free = [&](int w) { return bars + 8u * (3 + 4 * NS + w); };
+  auto p_full = [&](int w) { return bars + 8u * (5 + 4 * NS + w); };
+  auto pv_done = [&](int w) { return bars + 8u * (7 + 4 * NS + w); };
+  const uint32_t drain_bar = bars + 8u * (9 + 4 * NS);
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
+  volatile int* abort = misc + 1;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int qt = blockIdx.x, h = blockIdx.y;
+
+  if (tid == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(s_full(w), 1);
+      mbar_init(s_free(w), 128);
+      mbar_init(p_full(w), 128);
+      mbar_init(pv_done(w), 1);
+    }
+    mbar_init(drain_bar, 1);
+    fence_barrier_init();
+    misc[1] = 0;
+    if constexpr (DENSE) {
+      misc[2] = p.nkb;
+      misc[3] = 0;
+    } else {
+      const int* rp = p.row_ptr + static_cast<size_t>(h) * (p.nqb + 1);
+      const int st = rp[qt], en = rp[qt + 1];
+      int n = en - st;
+      if (st < 0 || n < 0 || n > p.nkb) {
+        n = 0;
+        if (p.err) atomicCAS(p.err, 0, kErrBadCsr);
+      }
+      misc[2] = n;
+      misc[3] = st;
+    }
+  }
+  if (warp == kDualKWarp) {
+    tmem_alloc(smem_u32(const_cast<int*>(misc)), C::TMEM_COLS);
+    tmem_relinquish();
+    if (lane == 0) {
+      tma_prefetch_map(&tmQ);
+      tma_prefetch_map(&tmK);
+      tma_prefetch_map(&tmV);
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+  const int nblk = misc[2];
+  const int csr_start = misc[3];
+  auto kb_at = [&](int j) -> int {
+    if constexpr (DENSE) {
+      return j;
+    } else {
+      return __ldg(p.col_idx + csr_start + j);
+    }
+  };
+
+  if (warp == kDualKWarp) {
+    // ===================================================== Q / K producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * (BM * 128), &tmQ, c * 64, qt * BM, h, bar_q);
+      int issued = 0;
+      for (int j = 0; j < nblk; ++j) {
+        const int s = j % NS;
+        if (!mbar_wait(k_empty(s), ((j / NS) & 1) ^ 1u, abort, p.err, kErrWaitKEmpty)) break;
+        mbar_arrive_expect_tx(k_full(s), C::KV_BYTES);
+        const int kb = kb_at(j);
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sK + s * C::KV_BYTES + c * (BK * 128), &tmK, c * 64, kb * BK, h, k_full(s));
+        issued = j + 1;
+      }
+      if (*abort) {
+        drain_wait(bar_q, 0);
+        for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
+          drain_wait(k_full(j % NS), (j / NS) & 1);
+      }
+    }
+  } else if (warp == kDualVWarp) {
+    // ===================================================== V producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int j = 0; j < nblk; ++j) {
+        const int s = j % NS;
+        if (!mbar_wait(v_empty(s), ((j / NS) & 1) ^ 1u, abort, p.err, kErrWaitVEmpty)) break;
+        mbar_arrive_expect_tx(v_full(s), C::KV_BYTES);
+        const int kb = kb_at(j);
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sV + s * C::KV_BYTES + c * (BK * 128), &tmV, c * 64, kb * BK, h, v_full(s));
+        issued = j + 1;
+      }
+      if (*abort) {
+        for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
+          drain_wait(v_full(j % NS), (j / NS) & 1);
+      }
+    }
+  } else if (warp == kDualMmaWarp) {
+    // ===================================================== MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BK, 0, 0);
+      constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, D, 0, 1);
+      auto qk_ready = [&](int j) -> bool {
+        const int s = j % NS, w = j & 1, i = j >> 1;
+        return mbar_test(k_full(s), (j / NS) & 1) && mbar_test(s_free(w), (i & 1) ^ 1u);
+      };
+      auto pv_ready = [&](int j) -> bool {
+        const int s = j % NS, w = j & 1, i = j >> 1;
+        return mbar_test(p_full(w), i & 1) && mbar_test(v_full(s), (j / NS) & 1);
+      };
+      auto issue_qk = [&](int j) {
+        const int s = j % NS, w = j & 1;
+        tc_fence_after();
+        const uint32_t tS = tmem + w * BK;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t a = smem_desc_sw128(sQ + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              smem_desc_sw128(sK + s * C::KV_BYTES + (k >> 2) * (BK * 128) + (k & 3) * 32, 16, 1024);
+          mma_bf16_ss(tS, a, bd, kIdescQK, k > 0 ? 1u : 0u);
+        }
+        mma_commit(k_empty(s));
+        mma_commit(s_full(w));
+      };
+      auto issue_pv = [&](int j) {
+        const int s = j % NS, w = j & 1, i = j >> 1;
+        tc_fence_after();
+        const uint32_t tO = tmem + 2 * BK + w * D;
+        const uint32_t pw = sP + w * C::P_BYTES;
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          const uint64_t a = smem_desc_sw128(pw + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024);
+          const uint64_t b = smem_desc_sw128(sV + s * C::KV_BYTES + k * 16 * 128, BK * 128, 1024);
+          mma_bf16_ss(tO, a, b, kIdescPV, (i > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(v_empty(s));
+        mma_commit(pv_done(w));
+      };
+      // Issue QK and PV in whatever order their inputs become ready, so that
+      // one warpgroup's softmax never holds back the other's next score tile.
+      // QK_j needs K_j and the release of S_{j mod 2} (block j-2); PV_j needs
+      // P_j and V_j.  Both streams stay in block order.
+      bool ok = mbar_wait(bar_q, 0, abort, p.err, kErrWaitQ);
+      int nq = 0, np = 0;
+      unsigned long long t_idle = 0;
+      int idle = 0;
+      while (ok && np < nblk) {
+        bool did = false;
+        if (nq < nblk && qk_ready(nq)) {
+          issue_qk(nq++);
+          did = true;
+        }
+        if (np < nq && pv_ready(np)) {
+          issue_pv(np++);
+          did = true;
+        }
+        if (did) {
+          idle = 0;
+        } else if (++idle == 1) {
+          t_idle = global_timer_ns();
+        } else if ((idle & 255) == 0) {
+          // nothing ready for a while: give up after the usual time limit
+          if (*abort) {
+            ok = false;
+          } else if (global_timer_ns() - t_idle > kWaitTimeoutNs) {
+            *abort = 1;
+            if (p.err) atomicCAS(p.err, 0, kErrWaitPFull);
+            ok = false;
+          }
+        }
+      }
+      if (!ok) {
+        mma_commit(drain_bar);
+        drain_wait(drain_bar, 0);
+      }
+    }
+  } else if (warp < 8) {
+    // ===================================================== softmax warpgroups (warps 0..7)
+    const int w = warp >> 2;                  // warpgroup 0 or 1
+    const int row = tid & 127;                // query row = TMEM lane
+    const uint32_t tl = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + tl + w * BK;
+    const uint32_t tO = tmem + tl + 2 * BK + w * D;
+    const uint32_t pw = sP + w * C::P_BYTES;
+    const int qpos = qt * BM + row;
+    const bool valid_row = qpos < p.N;
+    const int nmine = (nblk + 1 - w) >> 1;    // blocks of this warpgroup
+    float m_ref = -INFINITY, Z = 0.f, A = 0.f;
+    bool ok = true;
+    float sv[BK];
+    // P_w row `row`: 128-byte swizzled K-major rows, two 64-key halves of
+    // 128 rows each; chunk c8 (8 keys, 16 bytes) lands at prow + poff[c8]
+    const uint32_t prow = pw + row * 128;
+    uint32_t poff[BK / 8];
+#pragma unroll
+    for (int c8 = 0; c8 < BK / 8; ++c8) poff[c8] = (c8 >> 3) * (BM * 128) + (((c8 & 7) ^ (row & 7)) << 4);
+    for (int i = 0; i < nmine; ++i) {
+      const int j = 2 * i + w;
+      const int kb = kb_at(j);
+      ok = mbar_wait(s_full(w), i & 1, abort, p.err, kErrWaitSFull);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < BK / 32; ++c) tmem_ld32f(tS + c * 32, sv + c * 32);
+      tmem_wait_ld();
+      freg_fence<BK>(sv);
+      tc_fence_before();
+      mbar_arrive(s_free(w));   // S_w may now receive this warpgroup's next QK
+
+      int nvalid = p.N - kb * BK;
+      if constexpr (!DENSE) {
+        if (kb < 0 || kb >= p.nkb) nvalid = 0;
+      }
+      float alpha = 1.f;
+      bool o_rescale = false;
+      auto update_max = [&](float bmax) {
+        const float m_new = fmaxf(m_ref, bmax);
+        if (m_new > m_ref + kRescaleLog2) {
+          if (m_ref != -INFINITY) {
+            alpha = ex2_approx(m_ref - m_new);
+            A = alpha * (A + (m_ref - m_new) * Z);
+            Z *= alpha;
+            o_rescale = i > 0;
+          }
+          m_ref = m_new;
+        }
+      };
+      // Three cases, warp-uniform: every key of the block valid for the whole
+      // warp (fast path), none valid (P = 0), or a partly valid tail block.
+      const int mode = __all_sync(0xffffffffu, nvalid >= BK) ? 0
+                       : (__all_sync(0xffffffffu, nvalid <= 0) ? 1 : 2);
+      auto wait_prev_pv = [&]() -> bool {
+        // P_w and O_w are free once this warpgroup's previous PV has completed
+        if (i > 0) {
+          const bool done = mbar_wait(pv_done(w), (i - 1) & 1, abort, p.err, kErrWaitPVDone);
+          if (!__all_sync(0xffffffffu, done)) return false;
+        }
+        tc_fence_after();
+        return true;
+      };
+      auto rescale_o = [&]() {
+        if (__any_sync(0xffffffffu, o_rescale)) {
+          const float a = o_rescale ? alpha : 1.f;
+#pragma unroll
+          for (int c = 0; c < D; c += 16) {
+            float o[16];
+            tmem_ld16f(tO + c, o);
+            tmem_wait_ld();
+            freg_fence<16>(o);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] *= a;
+            tmem_st16f(tO + c, o);
+          }
+          tmem_wait_st();
+        }
+      };
+      if (mode == 1) {
+        // no key of this block is valid: P = 0, statistics unchanged
+        if (!wait_prev_pv()) { ok = false; break; }
+#pragma unroll
+        for (int c8 = 0; c8 < BK / 8; ++c8) st_shared_v4(prow + poff[c8], 0u, 0u, 0u, 0u);
+      } else {
+        if (mode == 2) {
+          // tail block: keys past N get a huge negative score, so p = 0 and
+          // p * x = 0 without special cases (at least one key is valid)
+#pragma unroll
+          for (int c = 0; c < BK; ++c) sv[c] = c < nvalid ? sv[c] : -1e30f;
+        }
+        {
+          // row max: 16 independent chains of 3-input max, then a small tree
+          float mx[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            mx[q] = fmax3(sv[q], sv[16 + q], sv[32 + q]);
+            mx[q] = fmax3(mx[q], sv[48 + q], sv[64 + q]);
+            mx[q] = fmax3(mx[q], sv[80 + q], sv[96 + q]);
+            mx[q] = fmaxf(mx[q], sv[112 + q]);
+          }
+#pragma unroll
+          for (int q = 0; q < 5; ++q) mx[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
+          const float m6 = fmax3(mx[0], mx[1], mx[2]);
+          const float m7 = fmax3(mx[3], mx[4], mx[15]);
+          update_max(fmaxf(m6, m7) * p.scale_log2);
+        }
+        // m_ref is finite here.  x = s * scale * log2(e) - m_ref, p = 2^x,
+        // Z += p, A += p * x, two lanes per instruction.
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(-m_ref, -m_ref);
+        float2 z2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        auto pair = [&](int c) -> uint32_t {
+          const float2 x = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nm2);
+          const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          z2[c & 1] = __fadd2_rn(z2[c & 1], pr);
+          if constexpr (DENSE) a2[c & 1] = __ffma2_rn(pr, x, a2[c & 1]);
+          return pack_bf16(pr.x, pr.y);
+        };
+        // the first half of the keys into registers while this warpgroup's
+        // previous PV (which reads P_w) finishes on the tensor cores
+        uint32_t first[BK / 4];
+#pragma unroll
+        for (int c = 0; c < BK / 4; ++c) first[c] = pair(c);
+        if (!wait_prev_pv()) { ok = false; break; }
+        rescale_o();
+#pragma unroll
+        for (int c8 = 0; c8 < BK / 16; ++c8)
+          st_shared_v4(prow + poff[c8], first[4 * c8], first[4 * c8 + 1], first[4 * c8 + 2],
+                       first[4 * c8 + 3]);
+        // the rest: computed and stored 8 keys at a time
+#pragma unroll
+        for (int c8 = BK / 16; c8 < BK / 8; ++c8) {
+          const uint32_t a = pair(4 * c8), b = pair(4 * c8 + 1);
+          const uint32_t c = pair(4 * c8 + 2), d = pair(4 * c8 + 3);
+          st_shared_v4(prow + poff[c8], a, b, c, d);
+        }
+        const float2 zz = __fadd2_rn(z2[0], z2[1]);
+        Z += zz.x + zz.y;
+        if constexpr (DENSE) {
+          const float2 aa = __fadd2_rn(a2[0], a2[1]);
+          A += aa.x + aa.y;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full(w));
+    }
+    // ---- merge the two warpgroups' partial results
+    if (ok && nmine > 0) {
+      ok = mbar_wait(pv_done(w), (nmine - 1) & 1, abort, p.err, kErrWaitPVDone);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    float* st = reinterpret_cast<float*>(smem + C::OFF_P + w * C::P_BYTES);  // P_w is free now
+    st[row] = m_ref;
+    st[128 + row] = Z;
+    st[256 + row] = A;
+    tc_fence_before();
+    named_barrier_sync(1, 256);
+    tc_fence_after();
+    const float* so = reinterpret_cast<const float*>(smem + C::OFF_P + (1 - w) * C::P_BYTES);
+    const float m_o = so[row], Z_o = so[128 + row], A_o = so[256 + row];
+    const float m0 = w == 0 ? m_ref : m_o, m1 = w == 0 ? m_o : m_ref;
+    const float Z0 = w == 0 ? Z : Z_o, Z1 = w == 0 ? Z_o : Z;
+    const float A0 = w == 0 ? A : A_o, A1 = w == 0 ? A_o : A;
+    const float m = fmaxf(m0, m1);
+    const float a0 = (m0 == -INFINITY) ? 0.f : ex2_approx(m0 - m);
+    const float a1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - m);
+    const float Zt = a0 * Z0 + a1 * Z1;
+    float At = 0.f;
+    if (a0 > 0.f) At += a0 * (A0 + (m0 - m) * Z0);
+    if (a1 > 0.f) At += a1 * (A1 + (m1 - m) * Z1);
+    const float inv = Zt > 0.f ? 1.f / Zt : 0.f;
+    const int n0 = (nblk + 1) >> 1, n1 = nblk >> 1;
+    const bool use0 = ok && n0 > 0, use1 = ok && n1 > 0;
+    const float c0 = use0 ? a0 * inv : 0.f, c1 = use1 ? a1 * inv : 0.f;
+    __nv_bfloat16* orow = p.O + (static_cast<size_t>(h) * p.N + (valid_row ? qpos : 0)) * D;
+    // warpgroup w writes output columns [w * D/2, (w + 1) * D/2)
+#pragma unroll
+    for (int c = w * (D / 2); c < (w + 1) * (D / 2); c += 16) {
+      float o0[16], o1[16];
+      if (use0) tmem_ld16f(tmem + tl + 2 * BK + c, o0);
+      if (use1) tmem_ld16f(tmem + tl + 2 * BK + D + c, o1);
+      tmem_wait_ld();
+      if (use0) freg_fence<16>(o0);
+      if (use1) freg_fence<16>(o1);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float x0 = use0 ? o0[e] * c0 : 0.f;
+        const float x1 = use1 ? o1[e] * c1 : 0.f;
+        o0[e] = x0 + x1;
+      }
+      if (valid_row) {
+        uint4 w0, w1;
+        w0.x = pack_bf16(o0[0], o0[1]);
+        w0.y = pack_bf16(o0[2], o0[3]);
+        w0.z = pack_bf16(o0[4], o0[5]);
+        w0.w = pack_bf16(o0[6], o0[7]);
+        w1.x = pack_bf16(o0[8], o0[9]);
+        w1.y = pack_bf16(o0[10], o0[11]);
+        w1.z = pack_bf16(o0[12], o0[13]);
+        w1.w = pack_bf16(o0[14], o0[15]);
+        reinterpret_cast<uint4*>(orow + c)[0] = w0;
+        reinterpret_cast<uint4*>(orow + c)[1] = w1;
+      }
+    }
+    if (w == 0 && valid_row) {
+      const size_t idx = static_cast<size_t>(h) * p.N + qpos;
+      if (DENSE && p.H != nullptr) p.H[idx] = Zt > 0.f ? logf(Zt) - kLn2 * (At / Zt) : NAN;
+      if (p.lse != nullptr) p.lse[idx] = Zt > 0.f ? kLn2 * (m + log2f(Zt)) : -INFINITY;
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == kDualKWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -611,6 +1118,21 @@ bool make_map(CUtensorMap* map, const void* base, int d, int N, int heads, int r
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+template <int D, bool DENSE>
+cudaError_t launch_dual(const AttnArgs& a, const Params& prm, cudaStream_t stream) {
+  using C = DualCfg<D>;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.Q, D, a.N, a.heads, BM) || !make_map(&mk, a.K, D, a.N, a.heads, C::BK) ||
+      !make_map(&mv, a.V, D, a.N, a.heads, C::BK))
+    return cudaErrorInvalidValue;
+  auto kern = attn_dual_kernel<D, DENSE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((a.N + BM - 1) / BM, a.heads);
+  kern<<<grid, kDualThreads, C::SMEM, stream>>>(mq, mk, mv, prm);
+  return cudaGetLastError();
 }
 
 template <int D, int BK, bool DENSE>
@@ -646,9 +1168,16 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
   prm.H = a.H;
   prm.lse = a.lse;
   prm.err = device_error_word();
+  // 128-row query blocks with 128-key blocks (and the dense pass) use the
+  // two-warpgroup kernel; smaller blocks use the single-warpgroup kernel,
+  // which also merges the lists of several query blocks per CTA.
   if (a.dense) {
-    if (a.d == 128) return launch_cfg<128, 128, true>(a, prm, stream);
-    return launch_cfg<64, 128, true>(a, prm, stream);
+    if (a.d == 128) return launch_dual<128, true>(a, prm, stream);
+    return launch_dual<64, true>(a, prm, stream);
+  }
+  if (bq == 128 && bk == 128) {
+    if (a.d == 128) return launch_dual<128, false>(a, prm, stream);
+    return launch_dual<64, false>(a, prm, stream);
   }
   if (a.d == 128) {
     if (bk == 128) return launch_cfg<128, 128, false>(a, prm, stream);

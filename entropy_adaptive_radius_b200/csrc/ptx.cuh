@@ -67,16 +67,47 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits until the phase of `bar` with parity `parity` has completed.  Gives up
-// when another role of the CTA has set *abort, or after kWaitTimeoutNs; in the
-// latter case it sets *abort and records `code` in the device error word.
+// Non-blocking test of a phase (never suspends).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Longest hardware suspension of one try_wait (ns).  A suspended thread issues
+// no instructions; it resumes when the phase completes or the hint expires.
+constexpr uint32_t kSuspendHintNs = 20000;
+
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits until the phase of `bar` with parity `parity` has completed.  The
+// thread sleeps inside try_wait (so a waiting warp does not take issue slots
+// from the warps sharing its scheduler); between sleeps it gives up when
+// another role of the CTA has set *abort, or after kWaitTimeoutNs, in which
+// case it sets *abort and records `code` in the device error word.
 // Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           int* err, int code) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_sleep(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     if (*abort) return false;
     if (global_timer_ns() - t0 > kWaitTimeoutNs) {
       *abort = 1;
