@@ -109,6 +109,18 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(value_ms, device=None):
+    """Largest value over all ranks of the default process group (each rank
+    times its own work with CUDA events; the job is as slow as its slowest
+    rank).  Returns the value unchanged without a process group."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value_ms
+    t = torch.tensor([float(value_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def kept_pair_tokens(row_ptr, col_idx, heads, N, bq, bk):
     """sum over kept (qb, kb) of |qb| * |kb| (tail blocks shorter), all heads."""
     nqb, nkb = -(-N // bq), -(-N // bk)
@@ -335,9 +347,7 @@ def gpu_arm(args, rank, world, local):
     elapsed_ms = start.elapsed_time(stop)
     launches = pipe.launches
     if world > 1:
-        t = torch.tensor([elapsed_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+        elapsed_ms = max_over_ranks(elapsed_ms, device)
         dist.barrier()
     if tra.tra_get_device_error() != 0:
         raise RuntimeError("device-side wait timed out in the timed region")
@@ -457,9 +467,7 @@ def e2e_run(pipe, host, dev, calls, args, device, world):
     torch.cuda.synchronize()
     ms = s.elapsed_time(e)
     if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, device)
     return {"ms": ms / steps, "h2d": h2d // steps, "d2h": d2h // steps}
 
 

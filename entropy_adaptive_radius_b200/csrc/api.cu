@@ -228,6 +228,7 @@ tra_status tra_build_block_mask(const float* r, const float* phi, int heads, tra
   if (heads < 0 || !grid_ok(grid) || !tile_ok(tile)) return TRA_ERR_INVALID_ARGUMENT;
   if (!block_ok(block_q) || !block_ok(block_k)) return TRA_ERR_UNSUPPORTED;
   if (vote_threshold < 1) return TRA_ERR_INVALID_ARGUMENT;
+  if (grid.F > kMaxMaskFrames) return TRA_ERR_UNSUPPORTED;
   if (col_capacity < 0) return TRA_ERR_CAPACITY;
   if (nnz == nullptr) return TRA_ERR_INVALID_ARGUMENT;
   const long long N = static_cast<long long>(grid.F) * grid.H * grid.W;

@@ -121,27 +121,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for two lanes on the FMA pipe (Cody-Waite style reduction): x = n + f
-// with n = rint(x) (adding 1.5 * 2^23 leaves rint(x) in the low mantissa bits
-// of t), f in [-1/2, 1/2], 2^f from a degree-3 polynomial minimax in relative
-// error on that interval (max relative error 7.5e-5; coefficients fitted by
-// Remez exchange, see fit_exp2_poly.py), and 2^n applied by adding n to the
-// exponent field: bits(t) << 23 == n << 23 (mod 2^32).  x is clamped below at
-// -125 so the exponent stays in range; results there are below 2^-124.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
-  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-  float2 q = __ffma2_rn(f, make_float2(0.055171669f, 0.055171669f),
-                        make_float2(0.24261112f, 0.24261112f));
-  q = __ffma2_rn(q, f, make_float2(0.69326099f, 0.69326099f));
-  q = __ffma2_rn(q, f, make_float2(0.99992807f, 0.99992807f));
-  return make_float2(__int_as_float((__float_as_int(t.x) << 23) + __float_as_int(q.x)),
-                     __int_as_float((__float_as_int(t.y) << 23) + __float_as_int(q.y)));
-}
-
 __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float* v) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "

@@ -149,73 +149,36 @@ __global__ void footprint_kernel(TileLayout L, int bk, MaskWs ws) {
 
 // -------------------------------------------------------------------- 2. votes
 
-struct QueryInfo {
-  int x, y, t;
-  float r;
-};
-
-// Number of keys of key block `kb` inside the support of query q, or, when
-// `exists` is set, 1 if there is at least one and 0 otherwise.
-__device__ __forceinline__ int count_in_block(const QueryInfo& q, int kb, int bk, int nrows,
-                                              const uint2* __restrict__ rows, const float* s_phi,
-                                              const TileLayout& L, int N, bool exists) {
-  int cnt = 0;
-  if (nrows >= 0) {
-    for (int i = 0; i < nrows; ++i) {
-      const uint2 rw = rows[i];
-      const int t = static_cast<int>(rw.x >> 16);
-      const int y = static_cast<int>(rw.x & 0xFFFFu);
-      const int xlo = static_cast<int>(rw.y >> 16);
-      const int xhi = static_cast<int>(rw.y & 0xFFFFu);
-      const int dt = t > q.t ? t - q.t : q.t - t;
-      const int rsq = radius_sq(q.r, s_phi[dt]);
-      const int dy = y - q.y;
-      const int m = rsq - dy * dy;
-      if (m < 0) continue;
-      if (exists) {
-        const int dx = max(0, max(xlo - q.x, q.x - xhi));
-        if (dx * dx <= m) return 1;
-      } else {
-        const int s = isqrt_floor(m);
-        const int lo = max(xlo, q.x - s), hi = min(xhi, q.x + s);
-        if (hi >= lo) cnt += hi - lo + 1;
-      }
-    }
-  } else {
-    const int p1 = min(N, (kb + 1) * bk);
-    for (int p = kb * bk; p < p1; ++p) {
-      const Coord c = tile_major_coord(L, p);
-      const int dt = c.t > q.t ? c.t - q.t : q.t - c.t;
-      const int rsq = radius_sq(q.r, s_phi[dt]);
-      const int dx = c.x - q.x, dy = c.y - q.y;
-      if (dx * dx + dy * dy <= rsq) {
-        if (exists) return 1;
-        ++cnt;
-      }
-    }
-  }
-  return cnt;
-}
-
-// grid (nqb, heads), kVoteThreads threads.  Dynamic smem: 4*F ints (per-frame
-// union boxes of the disks).
+// grid (nqb, heads), kVoteThreads threads.  Dynamic smem: F * 128 ints
+// (floor of each query's fp32 squared radius in each key frame) + 4 * F ints
+// (per-frame union boxes of the disks).
+//
+// Exact phase: a warp takes one candidate key block; lane l holds queries
+// l, l+32, l+64, l+96; the warp walks the block's rows (t, y, [x_lo, x_hi])
+// and, per row, counts for each of its queries the keys of the row inside the
+// query's disk: with m = floor(R2) - dy^2 >= 0 they are the x in [x_lo, x_hi]
+// with (x - x_q)^2 <= m.  With a vote threshold of 1 only existence matters:
+// the nearest x of the row is tested, and the block is kept at the first row
+// where any query has a hit.
 __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __restrict__ r,
                                                              const float* __restrict__ phi,
                                                              TileLayout L, int bq, int bk, int vote,
                                                              MaskWs ws) {
-  extern __shared__ int s_box[];  // [4][F]: x_lo, x_hi, y_lo, y_hi
+  extern __shared__ int s_dyn[];
   __shared__ float s_phi[kMaxFrames];
-  __shared__ QueryInfo s_q[128];
+  __shared__ int s_qx[128], s_qy[128], s_qt[128];
+  __shared__ float s_qr[128];
   __shared__ int s_count;
   const int N = L.F * L.H * L.W;
   const MaskDims md = mask_dims(L, bq, bk);
   const int qb = blockIdx.x, h = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int F = L.F;
-  int* bxlo = s_box;
-  int* bxhi = s_box + F;
-  int* bylo = s_box + 2 * F;
-  int* byhi = s_box + 3 * F;
+  int* s_rsq = s_dyn;               // [F][128]
+  int* bxlo = s_dyn + F * 128;      // [F] each
+  int* bxhi = bxlo + F;
+  int* bylo = bxlo + 2 * F;
+  int* byhi = bxlo + 3 * F;
 
   for (int t = tid; t < F; t += kVoteThreads) {
     s_phi[t] = phi[t];
@@ -224,35 +187,53 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
   if (tid == 0) s_count = 0;
   const int q0 = qb * bq;
   const int nq = min(bq, N - q0);
-  if (tid < nq) {
-    const Coord c = tile_major_coord(L, q0 + tid);
-    float rv = r[static_cast<size_t>(h) * N + q0 + tid];
-    if (rv != rv) rv = __int_as_float(0x7f800000);  // NaN keeps every key, like +inf
-    s_q[tid] = QueryInfo{c.x, c.y, c.t, rv};
+  if (tid < 128) {
+    if (tid < nq) {
+      const Coord c = tile_major_coord(L, q0 + tid);
+      float rv = r[static_cast<size_t>(h) * N + q0 + tid];
+      if (rv != rv) rv = __int_as_float(0x7f800000);  // NaN keeps every key, like +inf
+      s_qx[tid] = c.x; s_qy[tid] = c.y; s_qt[tid] = c.t; s_qr[tid] = rv;
+    } else {
+      s_qx[tid] = 0; s_qy[tid] = 0; s_qt[tid] = 0; s_qr[tid] = 0.f;
+    }
   }
   __syncthreads();
 
-  // Per key frame: box containing every query's disk in that frame.
-  for (int t = 0; t < F; ++t) {
-    int xlo = INT_MAX, xhi = INT_MIN, ylo = INT_MAX, yhi = INT_MIN;
-    if (tid < nq) {
-      const QueryInfo q = s_q[tid];
-      const int dt = t > q.t ? t - q.t : q.t - t;
-      const int s = isqrt_floor(radius_sq(q.r, s_phi[dt]));
-      xlo = q.x - s; xhi = q.x + s; ylo = q.y - s; yhi = q.y + s;
-    }
-    xlo = __reduce_min_sync(0xffffffffu, xlo);
-    xhi = __reduce_max_sync(0xffffffffu, xhi);
-    ylo = __reduce_min_sync(0xffffffffu, ylo);
-    yhi = __reduce_max_sync(0xffffffffu, yhi);
-    if (lane == 0 && xlo != INT_MAX) {
-      atomicMin(&bxlo[t], xlo); atomicMax(&bxhi[t], xhi);
-      atomicMin(&bylo[t], ylo); atomicMax(&byhi[t], yhi);
+  // Per key frame: each query's integer threshold, and the box containing
+  // every query's disk in that frame.
+  {
+    const bool mine = tid < nq;
+    const int qx = s_qx[tid], qy = s_qy[tid], qt = s_qt[tid];
+    const float qr = s_qr[tid];
+    for (int t = 0; t < F; ++t) {
+      const int dt = t > qt ? t - qt : qt - t;
+      const int rsq = mine ? radius_sq(qr, s_phi[dt]) : -1;  // -1: no key ever inside
+      s_rsq[t * 128 + tid] = rsq;
+      int xlo = INT_MAX, xhi = INT_MIN, ylo = INT_MAX, yhi = INT_MIN;
+      if (mine) {
+        const int sq = isqrt_floor(rsq);
+        xlo = qx - sq; xhi = qx + sq; ylo = qy - sq; yhi = qy + sq;
+      }
+      xlo = __reduce_min_sync(0xffffffffu, xlo);
+      xhi = __reduce_max_sync(0xffffffffu, xhi);
+      ylo = __reduce_min_sync(0xffffffffu, ylo);
+      yhi = __reduce_max_sync(0xffffffffu, yhi);
+      if (lane == 0 && xlo != INT_MAX) {
+        atomicMin(&bxlo[t], xlo); atomicMax(&bxhi[t], xhi);
+        atomicMin(&bylo[t], ylo); atomicMax(&byhi[t], yhi);
+      }
     }
   }
   __syncthreads();
 
   const bool exists = (vote == 1);
+  // this lane's queries
+  int qx[4], qy[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    qx[k] = s_qx[lane + 32 * k];
+    qy[k] = s_qy[lane + 32 * k];
+  }
   uint32_t* bits_row = ws.bits + (static_cast<size_t>(h) * md.nqb + qb) * md.nkbw;
   int my_count = 0;
   for (int w = warp; w < md.nkbw; w += kVoteThreads / 32) {
@@ -275,22 +256,67 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
     }
     uint32_t cand = __ballot_sync(0xffffffffu, survive);
     uint32_t word = 0;
-    // exact votes, lanes over queries
+    // exact votes, lanes over queries, rows of the key block in turn
     while (cand) {
       const int b = __ffs(cand) - 1;
       cand &= cand - 1;
       const int kb2 = w * 32 + b;
       const int nrows = __shfl_sync(0xffffffffu, info.x, b);
-      const uint2* rows = ws.rows + static_cast<size_t>(kb2) * bk;
-      int votes = 0;
-      for (int base = 0; base < nq; base += 32) {
-        const int i = base + lane;
-        int c = 0;
-        if (i < nq) c = count_in_block(s_q[i], kb2, bk, nrows, rows, s_phi, L, N, exists);
-        votes += __reduce_add_sync(0xffffffffu, c);
-        if (votes >= vote) break;
+      bool keep = false;
+      if (nrows >= 0) {
+        const uint2* rows = ws.rows + static_cast<size_t>(kb2) * bk;
+        int votes = 0;
+        for (int i = 0; i < nrows; ++i) {
+          const uint2 rw = rows[i];
+          const int t = static_cast<int>(rw.x >> 16);
+          const int y = static_cast<int>(rw.x & 0xFFFFu);
+          const int xlo = static_cast<int>(rw.y >> 16);
+          const int xhi = static_cast<int>(rw.y & 0xFFFFu);
+          const int* rs = s_rsq + t * 128 + lane;
+          if (exists) {
+            bool hit = false;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int dy = y - qy[k];
+              const int m = rs[32 * k] - dy * dy;
+              const int dx = max(0, max(xlo - qx[k], qx[k] - xhi));
+              hit |= (m >= 0) & (dx * dx <= m);
+            }
+            if (__any_sync(0xffffffffu, hit)) { keep = true; break; }
+          } else {
+            int cnt = 0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int dy = y - qy[k];
+              const int m = rs[32 * k] - dy * dy;
+              if (m >= 0) {
+                const int sq = isqrt_floor(m);
+                const int lo = max(xlo, qx[k] - sq), hi = min(xhi, qx[k] + sq);
+                if (hi >= lo) cnt += hi - lo + 1;
+              }
+            }
+            votes += __reduce_add_sync(0xffffffffu, cnt);
+            if (votes >= vote) { keep = true; break; }
+          }
+        }
+      } else {
+        // key block whose rows are not contiguous: token by token
+        int votes = 0;
+        const int p1 = min(N, (kb2 + 1) * bk);
+        for (int pp = kb2 * bk; pp < p1 && !keep; ++pp) {
+          const Coord c = tile_major_coord(L, pp);
+          const int* rs = s_rsq + c.t * 128 + lane;
+          int cnt = 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int dx = c.x - qx[k], dy = c.y - qy[k];
+            cnt += (dx * dx + dy * dy <= rs[32 * k]) ? 1 : 0;
+          }
+          votes += __reduce_add_sync(0xffffffffu, cnt);
+          keep = votes >= vote;
+        }
       }
-      if (votes >= vote) word |= 1u << b;
+      if (keep) word |= 1u << b;
     }
     if (lane == 0) bits_row[w] = word;
     my_count += __popc(word);
@@ -394,7 +420,13 @@ cudaError_t launch_block_mask(const float* r, const float* phi, int heads, const
   footprint_kernel<<<(md.nkb + 127) / 128, 128, 0, stream>>>(L, block_k, ws);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  votes_kernel<<<dim3(md.nqb, heads), kVoteThreads, 4 * L.F * sizeof(int), stream>>>(
+  const size_t votes_smem = (static_cast<size_t>(L.F) * 128 + 4 * L.F) * sizeof(int);
+  if (votes_smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(votes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(votes_smem));
+    if (e != cudaSuccess) return e;
+  }
+  votes_kernel<<<dim3(md.nqb, heads), kVoteThreads, votes_smem, stream>>>(
       r, phi, L, block_q, block_k, vote, ws);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

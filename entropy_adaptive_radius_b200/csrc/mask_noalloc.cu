@@ -74,6 +74,7 @@ extern "C" tra_status tra_build_block_mask_noalloc(const float* r, const float* 
   auto block_ok = [](int b) { return b == 16 || b == 64 || b == 128; };
   if (!block_ok(block_q) || !block_ok(block_k)) return TRA_ERR_UNSUPPORTED;
   if (vote_threshold < 1) return TRA_ERR_INVALID_ARGUMENT;
+  if (grid.F > kMaxMaskFrames) return TRA_ERR_UNSUPPORTED;
   if (col_capacity < 0) return TRA_ERR_CAPACITY;
   if (nnz == nullptr) return TRA_ERR_INVALID_ARGUMENT;
   const long long N = static_cast<long long>(grid.F) * grid.H * grid.W;

@@ -10,6 +10,7 @@
 namespace tra {
 
 constexpr int kMaxFrames = 1024;   // phi / frame tables live in kernel parameters
+constexpr int kMaxMaskFrames = 384;  // the mask keeps a 128-query x F threshold table in smem
 constexpr int kMaxSide = 16384;    // H, W bound: squared distances stay below 2^30
 
 // Device error word of the current device (a module-scope __device__ int).

@@ -167,7 +167,8 @@ size_t tra_mask_workspace_size(int heads, tra_grid grid, tra_tile tile, int bloc
  *                first col_capacity entries (capacity h*nqb*nkb never overflows).
  *   workspace    >= tra_mask_workspace_size(...) bytes, 256-byte aligned.
  *   block_q, block_k in {16, 64, 128};  vote_threshold >= 1;  tile as given
- *   to tra_tile_major_permute;  F <= 1024;  H, W <= 16384.
+ *   to tra_tile_major_permute;  F <= 384 (TRA_ERR_UNSUPPORTED above);
+ *   H, W <= 16384.
  */
 tra_status tra_build_block_mask(const float* r, const float* phi, int heads, tra_grid grid,
                                 tra_tile tile, int block_q, int block_k, int vote_threshold,

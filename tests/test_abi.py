@@ -112,6 +112,9 @@ def test_radius_and_mask_validation(L):
     assert m(P, P, 40, G, T, 128, 128, 1, P, P, 100, P, P, ws - 1, S0) == WORKSPACE
     assert m(P, P, 40, G, T, 128, 128, 1, P, P, 100, P, ctypes.c_void_p(4096 + 128), ws, S0) == WORKSPACE
     assert m(None, P, 40, G, T, 128, 128, 1, P, P, 100, P, P, ws, S0) == INVALID
+    # the threshold table of the mask kernel holds at most 384 key frames
+    g400 = tra.Grid(400, 4, 4)
+    assert m(P, P, 2, g400, T, 16, 16, 1, P, P, 100, P, P, 1 << 30, S0) == UNSUPPORTED
 
 
 def test_workspace_size_grows_with_problem(L):
