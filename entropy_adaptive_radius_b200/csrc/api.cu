@@ -172,7 +172,9 @@ tra_status tra_block_sparse_attn(const void* Q, const void* K, const void* V, vo
   if (heads == 0 || N == 0) return TRA_OK;
   if (row_ptr == nullptr || col_idx == nullptr) return TRA_ERR_INVALID_ARGUMENT;
   const long long nkb = (N + block_k - 1) / block_k;
-  if (block_q < 128 && nkb > 1024) return TRA_ERR_UNSUPPORTED;
+  // 16-token blocks run on the kernel that merges up to eight query blocks'
+  // lists in shared memory (at most 1024 key blocks)
+  if (block_q < 128 && (block_q == 16 || block_k == 16) && nkb > 1024) return TRA_ERR_UNSUPPORTED;
   s = check_device();
   if (s != TRA_OK) return s;
   AttnArgs a{};

@@ -598,6 +598,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   A = sum_w a_w (A_w + (m_w - m) Z_w),      O = (a_0 O_0 + a_1 O_1) / Z.
 // Warps: 0..7 softmax, 8 Q/K producer (and tensor-memory allocation), 9 MMA,
 // 10 V producer.
+//
+// Key blocks of 64 tokens are taken two at a time: a "super-block" of 128
+// keys is the next two entries of the CTA's key-block list, each loaded into
+// half of a K/V stage (a missing second entry loads rows past N, which read as
+// zeros).  When query blocks have 64 rows the CTA's 128 rows hold two query
+// blocks; its list is the merge of their two CSR rows, and each row masks out
+// the entries its own query block does not keep.  Every role walks that merge
+// itself, in the same order.
 // ---------------------------------------------------------------------------
 
 constexpr int kDualThreads = 352;  // 11 warps
@@ -607,7 +615,7 @@ constexpr int kDualVWarp = 10;
 
 template <int D>
 struct DualCfg {
-  static constexpr int BK = 128;
+  static constexpr int BK = 128;  // keys per super-block
   static constexpr int NS = 2;
   static constexpr int KCH = D / 64;
   static constexpr int Q_BYTES = BM * D * 2;
@@ -632,7 +640,38 @@ __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-template <int D, bool DENSE>
+// Walks the ascending union of up to two CSR rows (a, b), one entry per call:
+// returns the key block (-1 once both rows are exhausted) and sets `mem` to
+// bit 0 if the entry is in row a, bit 1 if it is in row b.
+struct ListWalker {
+  const int* a;
+  const int* b;
+  int na, nb, ia, ib;
+  __device__ __forceinline__ int next(uint32_t& mem) {
+    const int va = ia < na ? __ldg(a + ia) : INT_MAX;
+    const int vb = ib < nb ? __ldg(b + ib) : INT_MAX;
+    if (va == INT_MAX && vb == INT_MAX) {
+      mem = 0u;
+      return -1;
+    }
+    if (va < vb) {
+      ++ia;
+      mem = 1u;
+      return va;
+    }
+    if (vb < va) {
+      ++ib;
+      mem = 2u;
+      return vb;
+    }
+    ++ia;
+    ++ib;
+    mem = 3u;
+    return va;
+  }
+};
+
+template <int D, int BKS, bool DENSE>
 __global__ void __launch_bounds__(kDualThreads, 1)
     attn_dual_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
@@ -640,6 +679,8 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   using C = DualCfg<D>;
   constexpr int NS = C::NS;
   constexpr int BK = C::BK;
+  constexpr int E = BK / BKS;  // list entries per super-block (1 or 2)
+  static_assert(BKS == 64 || BKS == 128, "key block size");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -683,19 +724,32 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     mbar_init(drain_bar, 1);
     fence_barrier_init();
     misc[1] = 0;
+    // misc[2] super-blocks, misc[3..6] start / length of CSR rows a and b
     if constexpr (DENSE) {
       misc[2] = p.nkb;
-      misc[3] = 0;
+      misc[3] = 0; misc[4] = p.nkb; misc[5] = 0; misc[6] = 0;
     } else {
       const int* rp = p.row_ptr + static_cast<size_t>(h) * (p.nqb + 1);
-      const int st = rp[qt], en = rp[qt + 1];
-      int n = en - st;
-      if (st < 0 || n < 0 || n > p.nkb) {
-        n = 0;
-        if (p.err) atomicCAS(p.err, 0, kErrBadCsr);
+      int st[2] = {0, 0}, n[2] = {0, 0};
+      for (int g = 0; g < p.G; ++g) {
+        const int qb = qt * p.G + g;
+        if (qb >= p.nqb) break;
+        st[g] = rp[qb];
+        n[g] = rp[qb + 1] - st[g];
+        if (st[g] < 0 || n[g] < 0 || n[g] > p.nkb) {
+          n[g] = 0;
+          if (p.err) atomicCAS(p.err, 0, kErrBadCsr);
+        }
       }
-      misc[2] = n;
-      misc[3] = st;
+      int total = n[0];
+      if (n[1] > 0) {
+        ListWalker wk{p.col_idx + st[0], p.col_idx + st[1], n[0], n[1], 0, 0};
+        uint32_t mem;
+        total = 0;
+        while (wk.next(mem) >= 0) ++total;
+      }
+      misc[2] = (total + E - 1) / E;
+      misc[3] = st[0]; misc[4] = n[0]; misc[5] = st[1]; misc[6] = n[1];
     }
   }
   if (warp == kDualKWarp) {
@@ -710,13 +764,17 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
-  const int nblk = misc[2];
-  const int csr_start = misc[3];
-  auto kb_at = [&](int j) -> int {
+  const int nblk = misc[2];  // super-blocks
+  // a walker over this CTA's key-block list (dense: 0 .. nkb-1)
+  auto make_walker = [&]() {
+    return ListWalker{p.col_idx + misc[3], p.col_idx + misc[5], misc[4], misc[6], 0, 0};
+  };
+  auto next_entry = [&](ListWalker& wk, int& dense_next, uint32_t& mem) -> int {
     if constexpr (DENSE) {
-      return j;
+      mem = 1u;
+      return dense_next < p.nkb ? dense_next++ : -1;
     } else {
-      return __ldg(p.col_idx + csr_start + j);
+      return wk.next(mem);
     }
   };
 
@@ -727,14 +785,22 @@ __global__ void __launch_bounds__(kDualThreads, 1)
 #pragma unroll
       for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * (BM * 128), &tmQ, c * 64, qt * BM, h, bar_q);
       int issued = 0;
+      ListWalker wk = make_walker();
+      int dn = 0;
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NS;
         if (!mbar_wait(k_empty(s), ((j / NS) & 1) ^ 1u, abort, p.err, kErrWaitKEmpty)) break;
         mbar_arrive_expect_tx(k_full(s), C::KV_BYTES);
-        const int kb = kb_at(j);
 #pragma unroll
-        for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d(sK + s * C::KV_BYTES + c * (BK * 128), &tmK, c * 64, kb * BK, h, k_full(s));
+        for (int e = 0; e < E; ++e) {
+          uint32_t mem;
+          const int kb = next_entry(wk, dn, mem);
+          const int row0 = kb >= 0 ? kb * BKS : p.N;  // past N: zeros
+#pragma unroll
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_3d(sK + s * C::KV_BYTES + c * (BK * 128) + e * BKS * 128, &tmK, c * 64, row0,
+                        h, k_full(s));
+        }
         issued = j + 1;
       }
       if (*abort) {
@@ -747,14 +813,22 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     // ===================================================== V producer
     if (lane == 0) {
       int issued = 0;
+      ListWalker wk = make_walker();
+      int dn = 0;
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NS;
         if (!mbar_wait(v_empty(s), ((j / NS) & 1) ^ 1u, abort, p.err, kErrWaitVEmpty)) break;
         mbar_arrive_expect_tx(v_full(s), C::KV_BYTES);
-        const int kb = kb_at(j);
 #pragma unroll
-        for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d(sV + s * C::KV_BYTES + c * (BK * 128), &tmV, c * 64, kb * BK, h, v_full(s));
+        for (int e = 0; e < E; ++e) {
+          uint32_t mem;
+          const int kb = next_entry(wk, dn, mem);
+          const int row0 = kb >= 0 ? kb * BKS : p.N;
+#pragma unroll
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_3d(sV + s * C::KV_BYTES + c * (BK * 128) + e * BKS * 128, &tmV, c * 64, row0,
+                        h, v_full(s));
+        }
         issued = j + 1;
       }
       if (*abort) {
@@ -861,9 +935,30 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     uint32_t poff[BK / 8];
 #pragma unroll
     for (int c8 = 0; c8 < BK / 8; ++c8) poff[c8] = (c8 >> 3) * (BM * 128) + (((c8 & 7) ^ (row & 7)) << 4);
+    // this thread's walk of the key-block list, and its query block within
+    // the CTA (rows 64g .. 64g+63 when two 64-row query blocks share it)
+    ListWalker wk = make_walker();
+    int dn = 0, sb_done = 0;
+    const uint32_t my_bit = (p.G == 2) ? (1u << (row >> 6)) : 1u;
     for (int i = 0; i < nmine; ++i) {
       const int j = 2 * i + w;
-      const int kb = kb_at(j);
+      // entries of super-block j (skipping the other warpgroup's)
+      int nv[E];
+      for (; sb_done < j; ++sb_done) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          uint32_t mem;
+          next_entry(wk, dn, mem);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        uint32_t mem;
+        const int kb = next_entry(wk, dn, mem);
+        const bool keep = kb >= 0 && kb < p.nkb && (mem & my_bit) != 0u;
+        nv[e] = keep ? min(BKS, p.N - kb * BKS) : 0;
+      }
+      ++sb_done;
       ok = mbar_wait(s_full(w), i & 1, abort, p.err, kErrWaitSFull);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -875,9 +970,12 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       tc_fence_before();
       mbar_arrive(s_free(w));   // S_w may now receive this warpgroup's next QK
 
-      int nvalid = p.N - kb * BK;
-      if constexpr (!DENSE) {
-        if (kb < 0 || kb >= p.nkb) nvalid = 0;
+      // key c of the super-block is valid for this row iff c - BKS*e < nv[e]
+      bool all_valid = true, any_valid = false;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        all_valid = all_valid && nv[e] >= BKS;
+        any_valid = any_valid || nv[e] > 0;
       }
       float alpha = 1.f;
       bool o_rescale = false;
@@ -895,8 +993,8 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       };
       // Three cases, warp-uniform: every key of the block valid for the whole
       // warp (fast path), none valid (P = 0), or a partly valid tail block.
-      const int mode = __all_sync(0xffffffffu, nvalid >= BK) ? 0
-                       : (__all_sync(0xffffffffu, nvalid <= 0) ? 1 : 2);
+      const int mode = __all_sync(0xffffffffu, all_valid) ? 0
+                       : (__all_sync(0xffffffffu, !any_valid) ? 1 : 2);
       auto wait_prev_pv = [&]() -> bool {
         // P_w and O_w are free once this warpgroup's previous PV has completed
         if (i > 0) {
@@ -929,10 +1027,12 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         for (int c8 = 0; c8 < BK / 8; ++c8) st_shared_v4(prow + poff[c8], 0u, 0u, 0u, 0u);
       } else {
         if (mode == 2) {
-          // tail block: keys past N get a huge negative score, so p = 0 and
-          // p * x = 0 without special cases (at least one key is valid)
+          // partly valid: invalid keys (past N, or not kept by this row's
+          // query block) get a huge negative score, so p = 0 and p * x = 0
+          // without special cases; a row with no valid key leaves its
+          // statistics alone (below)
 #pragma unroll
-          for (int c = 0; c < BK; ++c) sv[c] = c < nvalid ? sv[c] : -1e30f;
+          for (int c = 0; c < BK; ++c) sv[c] = (c % BKS) < nv[c / BKS] ? sv[c] : -1e30f;
         }
         {
           // row max: 16 independent chains of 3-input max, then a small tree
@@ -948,12 +1048,14 @@ __global__ void __launch_bounds__(kDualThreads, 1)
           for (int q = 0; q < 5; ++q) mx[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
           const float m6 = fmax3(mx[0], mx[1], mx[2]);
           const float m7 = fmax3(mx[3], mx[4], mx[15]);
-          update_max(fmaxf(m6, m7) * p.scale_log2);
+          if (any_valid) update_max(fmaxf(m6, m7) * p.scale_log2);
         }
-        // m_ref is finite here.  x = s * scale * log2(e) - m_ref, p = 2^x,
-        // Z += p, A += p * x, two lanes per instruction.
+        // x = s * scale * log2(e) - m_ref, p = 2^x, Z += p, A += p * x, two
+        // lanes per instruction (m_ref is -inf only for a row with no valid
+        // key yet, whose p are then all 0)
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-        const float2 nm2 = make_float2(-m_ref, -m_ref);
+        const float mc = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const float2 nm2 = make_float2(-mc, -mc);
         float2 z2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         auto pair = [&](int c) -> uint32_t {
@@ -1099,14 +1201,14 @@ bool make_map(CUtensorMap* map, const void* base, int d, int N, int heads, int r
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool DENSE>
+template <int D, int BKS, bool DENSE>
 cudaError_t launch_dual(const AttnArgs& a, const Params& prm, cudaStream_t stream) {
   using C = DualCfg<D>;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, a.Q, D, a.N, a.heads, BM) || !make_map(&mk, a.K, D, a.N, a.heads, C::BK) ||
-      !make_map(&mv, a.V, D, a.N, a.heads, C::BK))
+  if (!make_map(&mq, a.Q, D, a.N, a.heads, BM) || !make_map(&mk, a.K, D, a.N, a.heads, BKS) ||
+      !make_map(&mv, a.V, D, a.N, a.heads, BKS))
     return cudaErrorInvalidValue;
-  auto kern = attn_dual_kernel<D, DENSE>;
+  auto kern = attn_dual_kernel<D, BKS, DENSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const dim3 grid((a.N + BM - 1) / BM, a.heads);
@@ -1147,16 +1249,19 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
   prm.H = a.H;
   prm.lse = a.lse;
   prm.err = device_error_word();
-  // 128-row query blocks with 128-key blocks (and the dense pass) use the
-  // two-warpgroup kernel; smaller blocks use the single-warpgroup kernel,
-  // which also merges the lists of several query blocks per CTA.
+  // Query and key blocks of 64 or 128 tokens (and the dense pass) use the
+  // two-warpgroup kernel; 16-token blocks use the single-warpgroup kernel,
+  // which merges the lists of up to eight query blocks per CTA.
   if (a.dense) {
-    if (a.d == 128) return launch_dual<128, true>(a, prm, stream);
-    return launch_dual<64, true>(a, prm, stream);
+    if (a.d == 128) return launch_dual<128, 128, true>(a, prm, stream);
+    return launch_dual<64, 128, true>(a, prm, stream);
   }
-  if (bq == 128 && bk == 128) {
-    if (a.d == 128) return launch_dual<128, false>(a, prm, stream);
-    return launch_dual<64, false>(a, prm, stream);
+  if ((bq == 128 || bq == 64) && (bk == 128 || bk == 64)) {
+    if (a.d == 128)
+      return bk == 128 ? launch_dual<128, 128, false>(a, prm, stream)
+                       : launch_dual<128, 64, false>(a, prm, stream);
+    return bk == 128 ? launch_dual<64, 128, false>(a, prm, stream)
+                     : launch_dual<64, 64, false>(a, prm, stream);
   }
   if (a.d == 128) {
     if (bk == 128) return launch_cfg<128, 128, false>(a, prm, stream);

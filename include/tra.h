@@ -219,8 +219,9 @@ tra_status tra_build_block_mask_noalloc(const float* r, const float* phi, int he
  *   lse       [heads, N] fp32 natural-log sum of exponentials, or NULL.
  *   row_ptr, col_idx  CSR as written by tra_build_block_mask for the same
  *             heads, N, block_q, block_k (col_idx ascending, no repeats).
- *   d in {64, 128}; block_q, block_k in {16, 64, 128};  when block_q < 128,
- *   ceil(N / block_k) <= 1024.  scale > 0 and finite.
+ *   d in {64, 128}; block_q, block_k in {16, 64, 128};  when block_q < 128
+ *   and either block is 16 tokens, ceil(N / block_k) <= 1024.  scale > 0 and
+ *   finite.
  */
 tra_status tra_block_sparse_attn(const void* Q, const void* K, const void* V, void* O,
                                  float* lse, const int* row_ptr, const int* col_idx, int heads,

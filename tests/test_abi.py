@@ -92,8 +92,8 @@ def test_attention_validation(L):
     assert s(P, P, P, P, None, P, P, 2, 1000, 128, 32, 128, 0.1, S0) == UNSUPPORTED
     assert s(P, P, P, P, None, P, P, 2, 1000, 128, 128, 48, 0.1, S0) == UNSUPPORTED
     assert s(P, P, P, P, None, None, P, 2, 1000, 128, 128, 128, 0.1, S0) == INVALID
-    # query blocks below 128 rows merge lists of at most 1024 key blocks
-    assert s(P, P, P, P, None, P, P, 2, 64 * 1025, 128, 64, 64, 0.1, S0) == UNSUPPORTED
+    # 16-token query blocks merge lists of at most 1024 key blocks
+    assert s(P, P, P, P, None, P, P, 2, 64 * 1025, 128, 16, 64, 0.1, S0) == UNSUPPORTED
 
 
 def test_radius_and_mask_validation(L):
