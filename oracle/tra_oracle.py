@@ -37,6 +37,24 @@ reason, in the design notes of the repository):
      kept when its votes reach the vote threshold.
   R7 a kept block pair contributes every one of its tokens to the exact
      softmax; a query whose row keeps nothing gets O = 0 and LSE = -inf.
+
+Mask variants (the ablations of §4 "ablation study", and the static mask of
+"Radial Attention: O(n log n) Sparse Attention with Energy Decay for Long
+Video Generation", abstract), all through the same token mask and votes:
+  R12 shared budget (entropy mapping removed): every query of a head gets the
+      budget K_h = mean over the head's queries of tau * exp(H_i), so the
+      head's total budget is unchanged; the radius follows from K_h as in R4.
+  R13 1D distance (radius masking replaced by a 1D distance): the distance of
+      two tokens is the difference of their in-frame raster indices
+      n = y * W + x; a key is inside when (n_j - n_i)^2 <= R^2 with R as in R5;
+      the budget becomes a radius by equal length,
+      K_i = 2 r_i * sum_t' phi(|t' - t_i|).
+  R14 Radial's static window: every query has the same base radius r0 (no
+      entropy), and the decay table is phi_R(delta) = 2^(-b/2) for the disk
+      (2^(-b) for the 1D distance) with b = floor(log2(delta + 1)): each time
+      the temporal distance doubles the window's area (length) halves, so every
+      band of temporal distances holds the same number of keys and a query's
+      support grows with log F (the O(n log n) cost the Radial page states).
 """
 import math
 
@@ -183,25 +201,85 @@ def radius(H, frame_of_query, tau, gamma, F, N):
 
 
 # ---------------------------------------------------------------------------
-# token mask, block votes, block mask, CSR  (§2 pipeline, fused mask kernel;
-# readings R5, R6)
+# mask variants: shared budget, 1D distance, Radial's static window
+# (§4 ablation study; Radial abstract; readings R12-R14)
 # ---------------------------------------------------------------------------
 
 
-def token_mask(r32, phi32, cq, ck):
-    """M[i, j] = 1 when key j lies in query i's disk of its frame.
+def shared_budget_tokens(H, tau):
+    """K_h = mean over the queries of head h of tau * exp(H_i)  (R12).
+    H: [heads, N]; returns [heads]."""
+    return np.mean(tau * np.exp(np.asarray(H, np.float64)), axis=1)
+
+
+def frame_length(F, gamma):
+    """L[t] = sum over existing key frames t' of phi(|t' - t|)  (R13)."""
+    L = np.zeros(F)
+    for t in range(F):
+        for tp in range(F):
+            L[t] += phi(abs(tp - t), gamma)
+    return L
+
+
+def radius_variant(H, frame_of_query, tau, gamma, F, budget="entropy", metric="disk"):
+    """Base radii [heads, N] of the budget source ("entropy": K_i = tau *
+    exp(H_i); "shared": K_h of R12 for every query of head h) and the distance
+    ("disk": r = sqrt(K / (pi S[t])), R4; "line": r = K / (2 L[t]), R13)."""
+    H = np.asarray(H, np.float64)
+    if budget == "entropy":
+        K = tau * np.exp(H)
+    elif budget == "shared":
+        K = np.repeat(shared_budget_tokens(H, tau)[:, None], H.shape[1], axis=1)
+    else:
+        raise ValueError(budget)
+    t = np.asarray(frame_of_query)
+    if metric == "disk":
+        return np.sqrt(K / (math.pi * frame_energy(F, gamma)[t]))
+    if metric == "line":
+        return K / (2.0 * frame_length(F, gamma)[t])
+    raise ValueError(metric)
+
+
+def radial_band(delta):
+    """b = floor(log2(delta + 1)) for integers delta >= 0."""
+    return np.array([int(dl + 1).bit_length() - 1 for dl in np.ravel(delta)], dtype=np.int64)
+
+
+def radial_phi(F, metric="disk"):
+    """Radial's window factor per temporal distance (R14): 2^(-b/2) for the
+    disk, 2^(-b) for the 1D distance, b = floor(log2(delta + 1))."""
+    b = radial_band(np.arange(F)).astype(np.float64)
+    return 2.0 ** (-b / 2.0) if metric == "disk" else 2.0 ** (-b)
+
+
+# ---------------------------------------------------------------------------
+# token mask, block votes, block mask, CSR  (§2 pipeline, fused mask kernel;
+# readings R5, R6, R13)
+# ---------------------------------------------------------------------------
+
+
+def token_mask(r32, phi32, cq, ck, metric="disk", W=None):
+    """M[i, j] = 1 when key j lies in query i's support in its frame.
 
     r32: float32 [Nq] base radii; phi32: float32 [F] decay table indexed by
     |t_j - t_i|; cq, ck: int [Nq, 3] / [Nk, 3] (x, y, t).  The threshold is
-    R2 = fl32(fl32(r * phi)^2); +inf or NaN radii keep every key."""
+    R2 = fl32(fl32(r * phi)^2); +inf or NaN radii keep every key.  metric
+    "disk": squared distance dx^2 + dy^2; "line" (R13): (n_j - n_i)^2 with the
+    in-frame raster index n = y * W + x."""
     r32 = np.asarray(r32, np.float32)
     phi32 = np.asarray(phi32, np.float32)
-    dx = cq[:, None, 0] - ck[None, :, 0]
-    dy = cq[:, None, 1] - ck[None, :, 1]
+    if metric == "disk":
+        dx = cq[:, None, 0] - ck[None, :, 0]
+        dy = cq[:, None, 1] - ck[None, :, 1]
+        d2 = (dx * dx + dy * dy).astype(np.float64)
+    elif metric == "line":
+        dn = (cq[:, None, 1] * W + cq[:, None, 0]) - (ck[None, :, 1] * W + ck[None, :, 0])
+        d2 = (dn * dn).astype(np.float64)
+    else:
+        raise ValueError(metric)
     dt = np.abs(cq[:, None, 2] - ck[None, :, 2])
     R = (r32[:, None] * phi32[dt]).astype(np.float32)      # fp32 product
     R2 = (R * R).astype(np.float32)                         # fp32 square
-    d2 = (dx * dx + dy * dy).astype(np.float64)
     keep_all = ~np.isfinite(r32)
     with np.errstate(invalid="ignore"):
         inside = d2 <= R2.astype(np.float64)
@@ -227,7 +305,8 @@ def block_mask_from_votes(votes, vote_threshold):
     return votes >= vote_threshold
 
 
-def block_mask(r32, phi32, coords_tm, Bq, Bk, vote_threshold, qblocks=None):
+def block_mask(r32, phi32, coords_tm, Bq, Bk, vote_threshold, qblocks=None, metric="disk",
+               W=None):
     """Kept-block mask of one head, bool [len(qblocks), nkb], brute force over
     every token pair.  coords_tm: (x, y, t) of each tile-major position."""
     N = coords_tm.shape[0]
@@ -238,7 +317,7 @@ def block_mask(r32, phi32, coords_tm, Bq, Bk, vote_threshold, qblocks=None):
     out = np.zeros((len(qblocks), nkb), dtype=bool)
     for row, qb in enumerate(qblocks):
         q = slice(qb * Bq, min(N, (qb + 1) * Bq))
-        M = token_mask(np.asarray(r32)[q], phi32, coords_tm[q], coords_tm)
+        M = token_mask(np.asarray(r32)[q], phi32, coords_tm[q], coords_tm, metric, W)
         out[row] = block_mask_from_votes(block_votes(M, Bq, Bk)[0], vote_threshold)
     return out
 
