@@ -165,11 +165,25 @@ class Pipeline:
         self.tau = 1.0
         self.vote = wl.vote
 
-    def mask(self, tau):
+    # mask source: ("entropy" | "shared" | "radial", "disk" | "line"); the
+    # parameter of mask() is tau for the entropy budgets and r0 for radial
+    variant = ("entropy", "disk")
+
+    def radius(self, param):
         w, t = self.wl, self.tra
-        t.tra_budget_radius(self.H, self.r, self.grid, tau, w.gamma, w.tile, phi_out=self.phi)
-        t.tra_build_block_mask(self.r, self.phi, self.grid, w.block_q, w.block_k, self.vote,
-                               self.row_ptr, self.col_idx, self.nnz, self.ws, w.tile)
+        source, metric = self.variant
+        if source == "radial":
+            t.tra_radial_radius(self.r, self.grid, param, metric, w.tile, phi_out=self.phi)
+        else:
+            t.tra_budget_radius_ex(self.H, self.r, self.grid, param, w.gamma, source, metric,
+                                   w.tile, phi_out=self.phi)
+
+    def mask(self, param):
+        w, t = self.wl, self.tra
+        self.radius(param)
+        t.tra_build_block_mask_ex(self.r, self.phi, self.grid, w.block_q, w.block_k, self.vote,
+                                  self.row_ptr, self.col_idx, self.nnz, self.ws, self.variant[1],
+                                  w.tile)
         self.launches += 5
 
     def warmup_call(self, Q, K, V, rec, out=None):
@@ -639,6 +653,51 @@ def sweep_arm(args):
             print(json.dumps(row), flush=True)
 
 
+def variants_arm(args):
+    """Mask variants at the 21x45x80, 40-head shape: TRA's per-query entropy
+    budget with the disk, the shared per-head budget (entropy mapping removed),
+    the 1D distance, and Radial Attention's static window (disk and 1D).  Each
+    variant's parameter (tau, or r0 for Radial) is bisected to the same kept
+    fraction as the bench's TRA workload; then its radius + mask time and the
+    block-sparse call over its CSR are timed.  One JSON line per variant."""
+    from entropy_adaptive_radius_b200 import tra
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    wl = workloads.WAN14B
+    log = lambda m: print(f"[variants] {m}", file=sys.stderr, flush=True)  # noqa: E731
+    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed, wl.q_scale, wl.dtype)
+    Qd, Kd, Vd = Q.to(device), K.to(device), V.to(device)
+    pipe = Pipeline(wl, device)
+    pipe.warmup_call(Qd, Kd, Vd, None)
+    torch.cuda.synchronize()
+    peaks, kind = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    for source, metric in (("entropy", "disk"), ("shared", "disk"), ("entropy", "line"),
+                           ("radial", "disk"), ("radial", "line")):
+        pipe.variant = (source, metric)
+        param = calibrate_tau(pipe, wl.kept_target, log)
+        pipe.mask(param)
+        kept = pipe.kept_fraction()
+        rp = pipe.row_ptr.cpu().numpy()
+        ci = pipe.col_idx[: int(pipe.nnz.item())].cpu().numpy()
+        pairs = kept_pair_tokens(rp, ci, wl.heads, wl.N, wl.block_q, wl.block_k)
+        ms = time_ms(lambda: tra.tra_block_sparse_attn(
+            pipe.Qtm, pipe.Ktm, pipe.Vtm, pipe.Otm, pipe.row_ptr, pipe.col_idx,
+            wl.block_q, wl.block_k), 5)
+        radius_ms = time_ms(lambda: pipe.radius(param), 5)
+        mask_ms = time_ms(lambda: pipe.mask(param), 5)
+        if tra.tra_get_device_error() != 0:
+            raise RuntimeError("device-side wait timed out")
+        tf = 4.0 * wl.d * pairs / (ms * 1e-3) / 1e12
+        print(json.dumps({
+            "workload": wl.name, "variant": {"budget": source, "metric": metric},
+            "param": {"r0" if source == "radial" else "tau": round(param, 8)},
+            "kept_fraction": round(kept, 4), "radius_ms": round(radius_ms, 4),
+            "radius_plus_mask_ms": round(mask_ms, 3), "sparse_ms": round(ms, 3),
+            "sparse_tflops_kept": round(tf, 1), "roofline_frac": round(tf / peak, 4),
+            "peak": f"{peak} TFLOP/s ({kind} bf16 sustained)"}), flush=True)
+
+
 def reference_arm(args, rank, world):
     if rank != 0:
         return
@@ -738,9 +797,9 @@ def main():
     ap.add_argument("--case", choices=["dense", "sparse", "mask", "permute"], default=None,
                     help="run one kernel on a small case (for profiler captures)")
     ap.add_argument("--reps", type=int, default=3)
-    ap.add_argument("--workload", default="wan14b", choices=sorted(WORKLOADS) + ["sweep"],
-                    help="wan14b (default, the headline step), wan13b, hunyuan, tiny, or the "
-                         "density sweep")
+    ap.add_argument("--workload", default="wan14b", choices=sorted(WORKLOADS) + ["sweep", "variants"],
+                    help="wan14b (default, the headline step), wan13b, hunyuan, tiny, the "
+                         "density sweep, or the mask variants")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
@@ -755,6 +814,9 @@ def main():
         return
     if args.workload == "sweep":
         sweep_arm(args)
+        return
+    if args.workload == "variants":
+        variants_arm(args)
         return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -185,36 +185,92 @@ tra_status tra_block_sparse_attn(const void* Q, const void* K, const void* V, vo
   return status_of(launch_attention(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-tra_status tra_budget_radius(const float* H, float* r, float* phi_out, int heads, tra_grid grid,
-                             tra_tile tile, float tau, float gamma, tra_stream_t stream) {
+tra_status tra_budget_radius_ex(const float* H, float* r, float* phi_out, int heads,
+                                tra_grid grid, tra_tile tile, float tau, float gamma,
+                                tra_budget budget, tra_metric metric, tra_stream_t stream) {
   if (heads < 0 || !grid_ok(grid) || !tile_ok(tile)) return TRA_ERR_INVALID_ARGUMENT;
   if (!(tau >= 0.f) || !std::isfinite(tau) || !(gamma >= 0.f) || !std::isfinite(gamma))
     return TRA_ERR_INVALID_ARGUMENT;
+  if (budget != TRA_BUDGET_ENTROPY && budget != TRA_BUDGET_SHARED) return TRA_ERR_INVALID_ARGUMENT;
+  if (metric != TRA_METRIC_DISK && metric != TRA_METRIC_LINE) return TRA_ERR_INVALID_ARGUMENT;
   const long long N = static_cast<long long>(grid.F) * grid.H * grid.W;
   if (N == 0) return TRA_OK;
   if (heads == 0 && phi_out == nullptr) return TRA_OK;
   if (heads > 0 && (H == nullptr || r == nullptr)) return TRA_ERR_INVALID_ARGUMENT;
+  if (heads > 65535) return TRA_ERR_UNSUPPORTED;
   const tra_status dv = check_device();
   if (dv != TRA_OK) return dv;
-  // phi(delta) = exp(-gamma delta); S(t) = sum_t' phi(|t'-t|)^2;
-  // coef(t) = sqrt(tau / (pi S(t))) -- all in double, rounded once.
-  static thread_local FrameTables tab;
+  const bool line = metric == TRA_METRIC_LINE;
+  // phi(delta) = exp(-gamma delta); per query frame t the disk uses
+  // S(t) = sum_t' phi(|t'-t|)^2 and the 1D distance L(t) = sum_t' phi(|t'-t|);
+  // all in double, rounded once.
   const int F = grid.F;
   double phid[kMaxFrames];
-  for (int k = 0; k < F; ++k) {
-    phid[k] = std::exp(-static_cast<double>(gamma) * k);
-    tab.phi[k] = static_cast<float>(phid[k]);
-  }
+  double per_frame[kMaxFrames];  // 1 / (pi S(t)) or 1 / (2 L(t))
+  for (int k = 0; k < F; ++k) phid[k] = std::exp(-static_cast<double>(gamma) * k);
   for (int t = 0; t < F; ++t) {
-    double S = 0.0;
+    double acc = 0.0;
     for (int tp = 0; tp < F; ++tp) {
       const double f = phid[tp > t ? tp - t : t - tp];
-      S += f * f;
+      acc += line ? f : f * f;
     }
-    tab.coef[t] = static_cast<float>(std::sqrt(static_cast<double>(tau) / (M_PI * S)));
+    per_frame[t] = line ? 1.0 / (2.0 * acc) : 1.0 / (M_PI * acc);
   }
-  return status_of(launch_budget_radius(H, r, phi_out, heads, layout_of(grid, tile), tab,
-                                        reinterpret_cast<cudaStream_t>(stream)));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const TileLayout Lt = layout_of(grid, tile);
+  if (budget == TRA_BUDGET_ENTROPY) {
+    static thread_local FrameTables tab;
+    for (int k = 0; k < F; ++k) tab.phi[k] = static_cast<float>(phid[k]);
+    for (int t = 0; t < F; ++t) {
+      const double c = static_cast<double>(tau) * per_frame[t];
+      tab.coef[t] = static_cast<float>(line ? c : std::sqrt(c));
+    }
+    return status_of(launch_budget_radius(H, r, phi_out, heads, Lt, tab, line, st));
+  }
+  static thread_local FrameTablesD tabd;
+  for (int k = 0; k < F; ++k) tabd.phi[k] = static_cast<float>(phid[k]);
+  for (int t = 0; t < F; ++t) tabd.c[t] = per_frame[t];
+  if (heads == 0) {
+    // only the decay table is asked for
+    static thread_local FrameTables tab;
+    for (int k = 0; k < F; ++k) tab.phi[k] = tabd.phi[k];
+    return status_of(launch_fill_radius(nullptr, phi_out, 0, Lt, 0.f, tab, st));
+  }
+  return status_of(launch_shared_budget_radius(H, r, phi_out, heads, Lt, static_cast<double>(tau),
+                                               line, tabd, st));
+}
+
+tra_status tra_budget_radius(const float* H, float* r, float* phi_out, int heads, tra_grid grid,
+                             tra_tile tile, float tau, float gamma, tra_stream_t stream) {
+  return tra_budget_radius_ex(H, r, phi_out, heads, grid, tile, tau, gamma, TRA_BUDGET_ENTROPY,
+                              TRA_METRIC_DISK, stream);
+}
+
+tra_status tra_radial_radius(float* r, float* phi_out, int heads, tra_grid grid, tra_tile tile,
+                             float r0, tra_metric metric, tra_stream_t stream) {
+  if (heads < 0 || !grid_ok(grid) || !tile_ok(tile)) return TRA_ERR_INVALID_ARGUMENT;
+  if (!(r0 >= 0.f)) return TRA_ERR_INVALID_ARGUMENT;  // NaN and negative radii
+  if (metric != TRA_METRIC_DISK && metric != TRA_METRIC_LINE) return TRA_ERR_INVALID_ARGUMENT;
+  const long long N = static_cast<long long>(grid.F) * grid.H * grid.W;
+  if (N == 0) return TRA_OK;
+  if (heads == 0 && phi_out == nullptr) return TRA_OK;
+  if (heads > 0 && r == nullptr) return TRA_ERR_INVALID_ARGUMENT;
+  if (heads > 65535) return TRA_ERR_UNSUPPORTED;
+  const tra_status dv = check_device();
+  if (dv != TRA_OK) return dv;
+  // band b = floor(log2(delta + 1)); window factor 2^(-b/2) (disk: the area
+  // halves per band) or 2^(-b) (1D: the length halves per band)
+  static thread_local FrameTables tab;
+  for (int k = 0; k < grid.F; ++k) {
+    int b = 0;
+    while ((static_cast<unsigned>(k) + 1u) >> (b + 1)) ++b;
+    const double f = metric == TRA_METRIC_LINE ? std::ldexp(1.0, -b) : std::pow(2.0, -0.5 * b);
+    tab.phi[k] = static_cast<float>(f);
+    tab.coef[k] = 0.f;
+  }
+  return status_of(launch_fill_radius(heads > 0 ? r : nullptr, phi_out, heads,
+                                      layout_of(grid, tile), r0, tab,
+                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t tra_mask_workspace_size(int heads, tra_grid grid, tra_tile tile, int block_q, int block_k) {
@@ -223,11 +279,13 @@ size_t tra_mask_workspace_size(int heads, tra_grid grid, tra_tile tile, int bloc
   return mask_workspace_bytes(heads, layout_of(grid, tile), block_q, block_k);
 }
 
-tra_status tra_build_block_mask(const float* r, const float* phi, int heads, tra_grid grid,
-                                tra_tile tile, int block_q, int block_k, int vote_threshold,
-                                int* row_ptr, int* col_idx, long long col_capacity, int* nnz,
-                                void* workspace, size_t workspace_bytes, tra_stream_t stream) {
+tra_status tra_build_block_mask_ex(const float* r, const float* phi, int heads, tra_grid grid,
+                                   tra_tile tile, int block_q, int block_k, int vote_threshold,
+                                   tra_metric metric, int* row_ptr, int* col_idx,
+                                   long long col_capacity, int* nnz, void* workspace,
+                                   size_t workspace_bytes, tra_stream_t stream) {
   if (heads < 0 || !grid_ok(grid) || !tile_ok(tile)) return TRA_ERR_INVALID_ARGUMENT;
+  if (metric != TRA_METRIC_DISK && metric != TRA_METRIC_LINE) return TRA_ERR_INVALID_ARGUMENT;
   if (!block_ok(block_q) || !block_ok(block_k)) return TRA_ERR_UNSUPPORTED;
   if (vote_threshold < 1) return TRA_ERR_INVALID_ARGUMENT;
   if (grid.F > kMaxMaskFrames) return TRA_ERR_UNSUPPORTED;
@@ -255,8 +313,17 @@ tra_status tra_build_block_mask(const float* r, const float* phi, int heads, tra
   const tra_status dv = check_device();
   if (dv != TRA_OK) return dv;
   return status_of(launch_block_mask(r, phi, heads, layout_of(grid, tile), block_q, block_k,
-                                     vote_threshold, row_ptr, col_idx, col_capacity, nnz,
-                                     workspace, st));
+                                     vote_threshold, metric == TRA_METRIC_LINE, row_ptr,
+                                     col_idx, col_capacity, nnz, workspace, st));
+}
+
+tra_status tra_build_block_mask(const float* r, const float* phi, int heads, tra_grid grid,
+                                tra_tile tile, int block_q, int block_k, int vote_threshold,
+                                int* row_ptr, int* col_idx, long long col_capacity, int* nnz,
+                                void* workspace, size_t workspace_bytes, tra_stream_t stream) {
+  return tra_build_block_mask_ex(r, phi, heads, grid, tile, block_q, block_k, vote_threshold,
+                                 TRA_METRIC_DISK, row_ptr, col_idx, col_capacity, nnz, workspace,
+                                 workspace_bytes, stream);
 }
 
 tra_status tra_get_device_error(int* code, tra_stream_t stream) {

@@ -24,6 +24,13 @@
 //     once the threshold is reached (only "votes >= threshold" is needed).
 //  3. scan: exclusive prefix sum of the per-row kept counts -> row_ptr, nnz.
 //  4. compact: kept bits -> ascending col_idx.
+//
+// The 1D-distance variant (the ablation of the summary's §4 that replaces the
+// radius mask by a 1D distance) runs the same four launches: the distance of
+// two tokens of a frame is the difference of their raster indices
+// n = y * W + x, a key is inside when (n_j - n_i)^2 <= R2, and each query
+// keeps, per key frame, the index interval [n_i - s, n_i + s] with
+// s = isqrt(floor(R2)); boxes and rows are compared as index intervals.
 #include "tra_internal.h"
 
 namespace tra {
@@ -32,6 +39,7 @@ namespace {
 constexpr int kMaxSeg = 4;  // per-frame boxes kept per key block (more: no pruning)
 constexpr int kVoteThreads = 128;
 constexpr int kRsqCap = 1 << 30;
+constexpr int kReachCap = 1 << 30;  // 1D reach cap: beyond any in-frame index distance (< 2^24)
 
 struct MaskWs {
   uint2* rows;      // [nkb * Bk]: x = t << 16 | y, y = x_lo << 16 | x_hi
@@ -87,6 +95,19 @@ __device__ __forceinline__ int radius_sq(float r, float phi) {
   const float R2 = __fmul_rn(R, R);
   if (!(R2 < 1073741824.0f)) return kRsqCap;
   return __float2int_rz(R2);
+}
+
+// floor(sqrt(floor(fl32(fl32(r * phi)^2)))): the largest integer index
+// distance inside R, capped at 2^30 (also for +inf and NaN).
+__device__ __forceinline__ int line_reach(float r, float phi) {
+  const float R = __fmul_rn(r, phi);
+  const float R2 = __fmul_rn(R, R);
+  if (!(R2 < 1152921504606846976.0f)) return kReachCap;  // 2^60
+  const unsigned long long m = __float2ull_rz(R2);
+  unsigned long long sq = static_cast<unsigned long long>(sqrt(static_cast<double>(m)));
+  while (sq * sq > m) --sq;
+  while ((sq + 1) * (sq + 1) <= m) ++sq;
+  return sq > static_cast<unsigned long long>(kReachCap) ? kReachCap : static_cast<int>(sq);
 }
 
 // ---------------------------------------------------------------- 1. footprint
@@ -160,6 +181,13 @@ __global__ void footprint_kernel(TileLayout L, int bk, MaskWs ws) {
 // with (x - x_q)^2 <= m.  With a vote threshold of 1 only existence matters:
 // the nearest x of the row is tested, and the block is kept at the first row
 // where any query has a hit.
+//
+// LINE = true (1D distance): the table holds each query's reach s per key
+// frame, the per-frame "box" is the index interval [min(n - s), max(n + s)],
+// a key block's per-frame box becomes the index interval
+// [y_lo * W + x_lo, y_hi * W + x_hi] (a superset of its tokens' indices) and
+// a row (t, y, [x_lo, x_hi]) the interval [y W + x_lo, y W + x_hi].
+template <bool LINE>
 __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __restrict__ r,
                                                              const float* __restrict__ phi,
                                                              TileLayout L, int bq, int bk, int vote,
@@ -207,12 +235,21 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
     const float qr = s_qr[tid];
     for (int t = 0; t < F; ++t) {
       const int dt = t > qt ? t - qt : qt - t;
-      const int rsq = mine ? radius_sq(qr, s_phi[dt]) : -1;  // -1: no key ever inside
-      s_rsq[t * 128 + tid] = rsq;
       int xlo = INT_MAX, xhi = INT_MIN, ylo = INT_MAX, yhi = INT_MIN;
-      if (mine) {
-        const int sq = isqrt_floor(rsq);
-        xlo = qx - sq; xhi = qx + sq; ylo = qy - sq; yhi = qy + sq;
+      if constexpr (LINE) {
+        const int reach = mine ? line_reach(qr, s_phi[dt]) : -1;  // -1: no key ever inside
+        s_rsq[t * 128 + tid] = reach;
+        if (mine) {
+          const int qn = qy * L.W + qx;
+          xlo = qn - reach; xhi = qn + reach; ylo = 0; yhi = 0;
+        }
+      } else {
+        const int rsq = mine ? radius_sq(qr, s_phi[dt]) : -1;  // -1: no key ever inside
+        s_rsq[t * 128 + tid] = rsq;
+        if (mine) {
+          const int sq = isqrt_floor(rsq);
+          xlo = qx - sq; xhi = qx + sq; ylo = qy - sq; yhi = qy + sq;
+        }
       }
       xlo = __reduce_min_sync(0xffffffffu, xlo);
       xhi = __reduce_max_sync(0xffffffffu, xhi);
@@ -233,6 +270,7 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
   for (int k = 0; k < 4; ++k) {
     qx[k] = s_qx[lane + 32 * k];
     qy[k] = s_qy[lane + 32 * k];
+    if constexpr (LINE) qx[k] += qy[k] * L.W;  // raster index n = y W + x
   }
   uint32_t* bits_row = ws.bits + (static_cast<size_t>(h) * md.nqb + qb) * md.nkbw;
   int my_count = 0;
@@ -250,7 +288,12 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
         for (int i = 0; i < info.y && !survive; ++i) {
           const int4 s = sg[i];
           const int ylo = s.y >> 16, yhi = s.y & 0xFFFF, xlo = s.z >> 16, xhi = s.z & 0xFFFF;
-          survive = ylo <= byhi[s.x] && yhi >= bylo[s.x] && xlo <= bxhi[s.x] && xhi >= bxlo[s.x];
+          if constexpr (LINE) {
+            const int nlo = ylo * L.W + xlo, nhi = yhi * L.W + xhi;
+            survive = nlo <= bxhi[s.x] && nhi >= bxlo[s.x];
+          } else {
+            survive = ylo <= byhi[s.x] && yhi >= bylo[s.x] && xlo <= bxhi[s.x] && xhi >= bxlo[s.x];
+          }
         }
       }
     }
@@ -273,7 +316,31 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
           const int xlo = static_cast<int>(rw.y >> 16);
           const int xhi = static_cast<int>(rw.y & 0xFFFFu);
           const int* rs = s_rsq + t * 128 + lane;
-          if (exists) {
+          if constexpr (LINE) {
+            const int nlo = y * L.W + xlo, nhi = y * L.W + xhi;
+            if (exists) {
+              bool hit = false;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int reach = rs[32 * k];
+                const int dn = max(0, max(nlo - qx[k], qx[k] - nhi));
+                hit |= (reach >= 0) & (dn <= reach);
+              }
+              if (__any_sync(0xffffffffu, hit)) { keep = true; break; }
+            } else {
+              int cnt = 0;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int reach = rs[32 * k];
+                if (reach >= 0) {
+                  const int lo = max(nlo, qx[k] - reach), hi = min(nhi, qx[k] + reach);
+                  if (hi >= lo) cnt += hi - lo + 1;
+                }
+              }
+              votes += __reduce_add_sync(0xffffffffu, cnt);
+              if (votes >= vote) { keep = true; break; }
+            }
+          } else if (exists) {
             bool hit = false;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -309,8 +376,13 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
           int cnt = 0;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int dx = c.x - qx[k], dy = c.y - qy[k];
-            cnt += (dx * dx + dy * dy <= rs[32 * k]) ? 1 : 0;
+            if constexpr (LINE) {
+              const int dn = abs(c.y * L.W + c.x - qx[k]);
+              cnt += (rs[32 * k] >= 0 && dn <= rs[32 * k]) ? 1 : 0;
+            } else {
+              const int dx = c.x - qx[k], dy = c.y - qy[k];
+              cnt += (dx * dx + dy * dy <= rs[32 * k]) ? 1 : 0;
+            }
           }
           votes += __reduce_add_sync(0xffffffffu, cnt);
           keep = votes >= vote;
@@ -412,8 +484,9 @@ size_t mask_workspace_bytes(int heads, const TileLayout& L, int block_q, int blo
 }
 
 cudaError_t launch_block_mask(const float* r, const float* phi, int heads, const TileLayout& L,
-                              int block_q, int block_k, int vote, int* row_ptr, int* col_idx,
-                              long long capacity, int* nnz, void* workspace, cudaStream_t stream) {
+                              int block_q, int block_k, int vote, bool line, int* row_ptr,
+                              int* col_idx, long long capacity, int* nnz, void* workspace,
+                              cudaStream_t stream) {
   MaskWs ws;
   carve(L, heads, block_q, block_k, static_cast<char*>(workspace), &ws);
   const MaskDims md = mask_dims(L, block_q, block_k);
@@ -421,13 +494,14 @@ cudaError_t launch_block_mask(const float* r, const float* phi, int heads, const
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t votes_smem = (static_cast<size_t>(L.F) * 128 + 4 * L.F) * sizeof(int);
+  auto kernel = line ? votes_kernel<true> : votes_kernel<false>;
   if (votes_smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(votes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(votes_smem));
     if (e != cudaSuccess) return e;
   }
-  votes_kernel<<<dim3(md.nqb, heads), kVoteThreads, votes_smem, stream>>>(
-      r, phi, L, block_q, block_k, vote, ws);
+  kernel<<<dim3(md.nqb, heads), kVoteThreads, votes_smem, stream>>>(r, phi, L, block_q, block_k,
+                                                                    vote, ws);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   scan_kernel<<<1, kScanThreads, 0, stream>>>(heads, md.nqb, ws, row_ptr, nnz);

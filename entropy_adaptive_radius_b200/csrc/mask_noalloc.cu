@@ -108,6 +108,6 @@ extern "C" tra_status tra_build_block_mask_noalloc(const float* r, const float* 
   void* scratch = scratch_address();
   if (scratch == nullptr) return TRA_ERR_CUDA;
   const cudaError_t e = launch_block_mask(r, phi, heads, L, block_q, block_k, vote_threshold,
-                                          row_ptr, col_idx, col_capacity, nnz, scratch, st);
+                                          false, row_ptr, col_idx, col_capacity, nnz, scratch, st);
   return e == cudaSuccess ? TRA_OK : TRA_ERR_CUDA;
 }

@@ -23,18 +23,31 @@ cudaError_t launch_permute(const void* src, void* dst, tra_dtype in_dtype, tra_d
 
 // radius.cu
 struct FrameTables {
-  float coef[kMaxFrames];  // sqrt(tau / (pi * S(t))) per query frame t
-  float phi[kMaxFrames];   // exp(-gamma * delta)
+  float coef[kMaxFrames];  // per query frame t: sqrt(tau / (pi S(t))) (disk), tau / (2 L(t)) (1D)
+  float phi[kMaxFrames];   // decay table phi(delta)
 };
+struct FrameTablesD {
+  double c[kMaxFrames];   // per query frame t: 1 / (pi S(t)) (disk) or 1 / (2 L(t)) (1D)
+  float phi[kMaxFrames];  // decay table phi(delta)
+};
+// r = coef[t] * expf(e * H), e = 1/2 (disk) or 1 (1D distance)
 cudaError_t launch_budget_radius(const float* H, float* r, float* phi_out, int heads,
-                                 const TileLayout& L, const FrameTables& tables,
+                                 const TileLayout& L, const FrameTables& tables, bool line,
                                  cudaStream_t stream);
+// shared per-head budget K_h = tau * mean(exp(H)); r = sqrt(K_h c[t]) or K_h c[t]
+cudaError_t launch_shared_budget_radius(const float* H, float* r, float* phi_out, int heads,
+                                        const TileLayout& L, double tau, bool line,
+                                        const FrameTablesD& tables, cudaStream_t stream);
+// r = r0 everywhere; phi_out <- tables.phi
+cudaError_t launch_fill_radius(float* r, float* phi_out, int heads, const TileLayout& L, float r0,
+                               const FrameTables& tables, cudaStream_t stream);
 
 // mask.cu
 size_t mask_workspace_bytes(int heads, const TileLayout& L, int block_q, int block_k);
 cudaError_t launch_block_mask(const float* r, const float* phi, int heads, const TileLayout& L,
-                              int block_q, int block_k, int vote, int* row_ptr, int* col_idx,
-                              long long capacity, int* nnz, void* workspace, cudaStream_t stream);
+                              int block_q, int block_k, int vote, bool line, int* row_ptr,
+                              int* col_idx, long long capacity, int* nnz, void* workspace,
+                              cudaStream_t stream);
 
 // attention.cu
 struct AttnArgs {

@@ -18,6 +18,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtra.so")
 
 TRA_BF16, TRA_F32 = 0, 1
+TRA_METRIC_DISK, TRA_METRIC_LINE = 0, 1
+TRA_BUDGET_ENTROPY, TRA_BUDGET_SHARED = 0, 1
+METRICS = {"disk": TRA_METRIC_DISK, "line": TRA_METRIC_LINE}
+BUDGETS = {"entropy": TRA_BUDGET_ENTROPY, "shared": TRA_BUDGET_SHARED}
 STATUS = {0: "TRA_OK", 1: "TRA_ERR_INVALID_ARGUMENT", 2: "TRA_ERR_UNSUPPORTED",
           3: "TRA_ERR_WORKSPACE", 4: "TRA_ERR_CAPACITY", 5: "TRA_ERR_CUDA",
           6: "TRA_ERR_DEVICE", 7: "TRA_ERR_TIMEOUT"}
@@ -49,7 +53,12 @@ _PROTOS = {
     "tra_dense_attn_entropy": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                                         _c_float, _vp]),
     "tra_budget_radius": (_c_int, [_vp, _vp, _vp, _c_int, Grid, Tile, _c_float, _c_float, _vp]),
+    "tra_budget_radius_ex": (_c_int, [_vp, _vp, _vp, _c_int, Grid, Tile, _c_float, _c_float,
+                                      _c_int, _c_int, _vp]),
+    "tra_radial_radius": (_c_int, [_vp, _vp, _c_int, Grid, Tile, _c_float, _c_int, _vp]),
     "tra_mask_workspace_size": (_c_size, [_c_int, Grid, Tile, _c_int, _c_int]),
+    "tra_build_block_mask_ex": (_c_int, [_vp, _vp, _c_int, Grid, Tile, _c_int, _c_int, _c_int,
+                                         _c_int, _vp, _vp, _c_ll, _vp, _vp, _c_size, _vp]),
     "tra_build_block_mask": (_c_int, [_vp, _vp, _c_int, Grid, Tile, _c_int, _c_int, _c_int, _vp,
                                       _vp, _c_ll, _vp, _vp, _c_size, _vp]),
     "tra_build_block_mask_noalloc": (_c_int, [_vp, _vp, _c_int, Grid, Tile, _c_int, _c_int, _c_int,
@@ -158,6 +167,28 @@ def tra_budget_radius(H, r, grid, tau, gamma, tile=(1, 4, 4), phi_out=None, stre
     return r
 
 
+def tra_budget_radius_ex(H, r, grid, tau, gamma, budget="entropy", metric="disk", tile=(1, 4, 4),
+                         phi_out=None, stream=None):
+    """Base radii from the entropy with a choice of budget ("entropy" per query,
+    "shared" per head) and distance ("disk", "line")."""
+    _contig(H, r, phi_out)
+    heads = H.shape[0]
+    _check("tra_budget_radius_ex", lib().tra_budget_radius_ex(
+        _p(H), _p(r), _p(phi_out), heads, _grid(grid), _tile(tile), float(tau), float(gamma),
+        BUDGETS[budget], METRICS[metric], _stream(stream)))
+    return r
+
+
+def tra_radial_radius(r, grid, r0, metric="disk", tile=(1, 4, 4), phi_out=None, stream=None):
+    """Radial Attention's static window: r = r0 everywhere and the band table in phi_out."""
+    _contig(r, phi_out)
+    heads = r.shape[0]
+    _check("tra_radial_radius", lib().tra_radial_radius(
+        _p(r), _p(phi_out), heads, _grid(grid), _tile(tile), float(r0), METRICS[metric],
+        _stream(stream)))
+    return r
+
+
 def tra_mask_workspace_size(heads, grid, block_q, block_k, tile=(1, 4, 4)) -> int:
     return int(lib().tra_mask_workspace_size(heads, _grid(grid), _tile(tile), block_q, block_k))
 
@@ -171,6 +202,18 @@ def tra_build_block_mask(r, phi, grid, block_q, block_k, vote, row_ptr, col_idx,
     _check("tra_build_block_mask", lib().tra_build_block_mask(
         _p(r), _p(phi), heads, _grid(grid), _tile(tile), block_q, block_k, vote, _p(row_ptr),
         _p(col_idx), col_idx.numel(), _p(nnz), _p(workspace), workspace.numel(),
+        _stream(stream)))
+    return row_ptr, col_idx, nnz
+
+
+def tra_build_block_mask_ex(r, phi, grid, block_q, block_k, vote, row_ptr, col_idx, nnz,
+                            workspace, metric="disk", tile=(1, 4, 4), stream=None):
+    """tra_build_block_mask with a choice of distance ("disk" or "line")."""
+    _contig(r, phi, row_ptr, col_idx, nnz, workspace)
+    heads = r.shape[0]
+    _check("tra_build_block_mask_ex", lib().tra_build_block_mask_ex(
+        _p(r), _p(phi), heads, _grid(grid), _tile(tile), block_q, block_k, vote, METRICS[metric],
+        _p(row_ptr), _p(col_idx), col_idx.numel(), _p(nnz), _p(workspace), workspace.numel(),
         _stream(stream)))
     return row_ptr, col_idx, nnz
 

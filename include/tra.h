@@ -209,6 +209,76 @@ tra_status tra_build_block_mask_noalloc(const float* r, const float* phi, int he
                                         long long col_capacity, int* nnz, tra_stream_t stream);
 
 /*
+ * ---- Mask variants -------------------------------------------------------
+ * The ablations of the Token Radius Attention summary (§4 results, ablation
+ * study: the entropy-to-budget mapping removed, or the radius mask replaced
+ * by a 1D distance) and the static mask of "Radial Attention: O(n log n)
+ * Sparse Attention with Energy Decay for Long Video Generation" (abstract:
+ * each token attends to spatially nearby tokens, with a window that shrinks
+ * with temporal distance and a compute density that decays with it).  They
+ * differ from TRA only in where the radius comes from and in the distance;
+ * the votes, the CSR and the block-sparse attention are the same.
+ */
+typedef enum {
+  TRA_METRIC_DISK = 0, /* dx^2 + dy^2 in the frame (TRA's radius mask) */
+  TRA_METRIC_LINE = 1  /* (n_j - n_i)^2 with the in-frame raster index n = y * W + x */
+} tra_metric;
+
+typedef enum {
+  TRA_BUDGET_ENTROPY = 0, /* K_i = tau * exp(H_i): TRA's per-query budget */
+  TRA_BUDGET_SHARED = 1   /* K_h = mean over the head's queries of tau * exp(H_i),
+                             the same budget for every query of head h */
+} tra_budget;
+
+/*
+ * tra_budget_radius with a choice of budget and distance.
+ *   budget   TRA_BUDGET_ENTROPY: K_i = tau * exp(H_i) (tra_budget_radius).
+ *            TRA_BUDGET_SHARED: K_h = tau * (sum_i exp(H_i)) / N for every
+ *            query of head h, so the head's total budget is unchanged; the
+ *            sum runs in double in a fixed order, and each radius is
+ *            evaluated in double and rounded once.  One +inf entropy makes
+ *            the whole head's radii +inf, one NaN makes them NaN.
+ *   metric   TRA_METRIC_DISK: equal area, r = sqrt(K / (pi * S(t))),
+ *            S(t) = sum_t' phi(|t' - t|)^2 (as tra_budget_radius).
+ *            TRA_METRIC_LINE: equal length, the 1D windows of all key frames
+ *            hold K = 2 * r * L(t) tokens, L(t) = sum_t' phi(|t' - t|), so
+ *            r = K / (2 * L(t)).
+ * Everything else (layouts, phi_out, limits) is as for tra_budget_radius.
+ */
+tra_status tra_budget_radius_ex(const float* H, float* r, float* phi_out, int heads,
+                                tra_grid grid, tra_tile tile, float tau, float gamma,
+                                tra_budget budget, tra_metric metric, tra_stream_t stream);
+
+/*
+ * Radial Attention's static window as a radius source (no entropy).
+ *   r        [heads, N] fp32; written: r0 for every query.
+ *   phi_out  [F] fp32 or NULL: the window factor per temporal distance delta,
+ *            phi_R(delta) = 2^(-b/2) for TRA_METRIC_DISK and 2^(-b) for
+ *            TRA_METRIC_LINE, b = floor(log2(delta + 1)).  Each time the
+ *            temporal distance doubles, the window's area (length) halves, so
+ *            every band of temporal distances holds the same number of keys
+ *            and a query's support grows with log F.
+ *   r0 >= 0 (+inf keeps every key); F <= 1024.
+ * Feed r and phi_out to tra_build_block_mask_ex with the same metric.
+ */
+tra_status tra_radial_radius(float* r, float* phi_out, int heads, tra_grid grid, tra_tile tile,
+                             float r0, tra_metric metric, tra_stream_t stream);
+
+/*
+ * tra_build_block_mask with a choice of distance.  TRA_METRIC_DISK is
+ * tra_build_block_mask.  TRA_METRIC_LINE keeps key j for query i when
+ *     (n_j - n_i)^2 <= R2,  n = y * W + x,  R2 and R as for the disk,
+ * so in each key frame the query keeps the raster-index interval
+ * [n_i - s, n_i + s], s = floor(sqrt(floor(R2))), which runs across row
+ * ends.  Votes, CSR, workspace and limits are those of tra_build_block_mask.
+ */
+tra_status tra_build_block_mask_ex(const float* r, const float* phi, int heads, tra_grid grid,
+                                   tra_tile tile, int block_q, int block_k, int vote_threshold,
+                                   tra_metric metric, int* row_ptr, int* col_idx,
+                                   long long col_capacity, int* nnz, void* workspace,
+                                   size_t workspace_bytes, tra_stream_t stream);
+
+/*
  * Block-sparse attention over the kept blocks (§2 "TRA pipeline": the
  * block-sparse mask drives a block-sparse attention backend; reuse across
  * sparse steps).  Exact softmax over every token of the kept key blocks of

@@ -134,3 +134,24 @@ def test_valid_call_without_gpu_reports_device_error(L):
     assert L.tra_tile_major_permute(P, P2, 0, 0, 2, 128, G, T, S0) == DEVICE
     with pytest.raises(tra.TraError):
         tra._check("x", DEVICE)
+
+
+def test_variant_validation(L):
+    b = L.tra_budget_radius_ex
+    assert b(P, P, None, 2, G, T, 1.0, 0.3, 2, 0, S0) == INVALID       # unknown budget
+    assert b(P, P, None, 2, G, T, 1.0, 0.3, 0, 9, S0) == INVALID       # unknown metric
+    assert b(P, P, None, 2, G, T, -1.0, 0.3, 1, 1, S0) == INVALID
+    assert b(None, P, None, 2, G, T, 1.0, 0.3, 1, 0, S0) == INVALID
+    assert b(None, None, None, 0, G, T, 1.0, 0.3, 1, 1, S0) == OK
+    rr = L.tra_radial_radius
+    assert rr(P, None, 2, G, T, -1.0, 0, S0) == INVALID
+    assert rr(P, None, 2, G, T, float("nan"), 0, S0) == INVALID
+    assert rr(P, None, 2, G, T, 3.0, 4, S0) == INVALID
+    assert rr(None, None, 2, G, T, 3.0, 0, S0) == INVALID
+    assert rr(None, None, 0, G, T, 3.0, 1, S0) == OK
+    assert rr(P, None, 2, tra.Grid(2000, 2, 2), T, 3.0, 0, S0) == INVALID   # F > 1024
+    m = L.tra_build_block_mask_ex
+    ws = L.tra_mask_workspace_size(40, G, T, 128, 128)
+    assert m(P, P, 40, G, T, 128, 128, 1, 7, P, P, 100, P, P, ws, S0) == INVALID
+    assert m(P, P, 40, G, T, 128, 48, 1, 1, P, P, 100, P, P, ws, S0) == UNSUPPORTED
+    assert m(P, P, 40, G, T, 128, 128, 1, 1, P, P, 100, P, P, ws - 1, S0) == WORKSPACE
