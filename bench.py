@@ -698,6 +698,68 @@ def variants_arm(args):
             "peak": f"{peak} TFLOP/s ({kind} bf16 sustained)"}), flush=True)
 
 
+def reuse_arm(args):
+    """Cross-step reuse at the 21x45x80, 40-head shape: a 50-step denoising
+    run of one attention layer through the layer driver, for several reuse
+    policies (all steps dense; one dense warm-up then sparse; and entropy
+    refreshes every 10 steps, by an entropy-only pass or by a dense step).
+    Inputs stay on the GPU (the step's Q, K cycle through five perturbed
+    copies); each run is timed with CUDA events.  One JSON line per policy."""
+    from entropy_adaptive_radius_b200 import tra
+    from entropy_adaptive_radius_b200.layer import ReusePolicy, TraLayer
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    wl = workloads.WAN14B
+    log = lambda m: print(f"[reuse] {m}", file=sys.stderr, flush=True)  # noqa: E731
+    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed, wl.q_scale, wl.dtype)
+    seq = [(Q.to(device), K.to(device))]
+    for c in range(1, 5):
+        seq.append((inputs.perturb(Q, wl.seed, c, 0).to(device), inputs.perturb(K, wl.seed, c, 1).to(device)))
+    Vd = V.to(device)
+    pipe = Pipeline(wl, device)
+    pipe.warmup_call(seq[0][0], seq[0][1], Vd, None)
+    tau = calibrate_tau(pipe, wl.kept_target, log)
+    del pipe
+    steps = 50
+    policies = [("all dense", ReusePolicy(warmup=steps)),
+                ("warm-up 1, no refresh", ReusePolicy(warmup=1)),
+                ("warm-up 1, entropy-only refresh every 10", ReusePolicy(1, 10, "entropy")),
+                ("warm-up 1, dense refresh every 10", ReusePolicy(1, 10, "dense"))]
+    O_ = torch.empty_like(Vd)
+    # load every kernel once before any timing (the entropy-only one is first
+    # needed mid-run by the refresh policies)
+    tra.tra_attn_entropy(seq[0][0], seq[0][1],
+                         torch.empty(wl.heads, wl.N, dtype=torch.float32, device=device))
+    base = None
+    for name, pol in policies:
+        layer = TraLayer((wl.F, wl.H, wl.W), wl.heads, wl.d, tau=tau, gamma=wl.gamma, tile=wl.tile,
+                         block_q=wl.block_q, block_k=wl.block_k, vote=wl.vote, policy=pol,
+                         device=device)
+        for k in range(3):   # warm the kernels once (dense, sparse and refresh kinds)
+            layer(seq[0][0], seq[0][1], Vd, O_)
+        layer.reset()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for k in range(steps):
+            q, kk = seq[k % len(seq)]
+            layer(q, kk, Vd, O_)
+        e.record()
+        torch.cuda.synchronize()
+        if tra.tra_get_device_error() != 0:
+            raise RuntimeError("device-side wait timed out")
+        ms = s.elapsed_time(e)
+        base = ms if base is None else base
+        kinds = [pol.kind(k) for k in range(steps)]
+        print(json.dumps({
+            "workload": wl.name, "policy": name, "steps": steps,
+            "dense_steps": kinds.count("dense"), "entropy_only_refreshes": kinds.count("sparse+entropy"),
+            "tau": round(tau, 6), "kept_fraction_last_mask": round(int(layer.nnz.item()) / (wl.heads * layer.nqb * layer.nkb), 4),
+            "ms_per_run": round(ms, 2), "ms_per_step": round(ms / steps, 3),
+            "attention_speedup_vs_all_dense": round(base / ms, 3)}), flush=True)
+        del layer
+
+
 def reference_arm(args, rank, world):
     if rank != 0:
         return
@@ -728,7 +790,8 @@ def reference_arm(args, rank, world):
 
 def kernel_case(args):
     """Small single-kernel cases for profiler captures (inputs > L2, < 1 GB):
-    dense / sparse: 40 heads x 16384 tokens x d=128 bf16 (168 MB per tensor);
+    dense / sparse / entropy (entropy only, no PV): 40 heads x 16384 tokens x
+    d=128 bf16 (168 MB per tensor);
     mask: the 21x45x80 grid, 40 heads, radii from entropies near ln N;
     permute: one 21x45x80 x 40-head x 128 bf16 tensor.  Runs the kernel
     `--reps` times and prints the mean CUDA-event time per launch."""
@@ -738,7 +801,7 @@ def kernel_case(args):
     g = torch.Generator(device=dev).manual_seed(0)
     heads, N, d = 40, 16384, 128
     reps = args.reps
-    if args.case in ("dense", "sparse"):
+    if args.case in ("dense", "sparse", "entropy"):
         Q = (torch.randn(heads, N, d, generator=g, device=dev) * 2).to(torch.bfloat16)
         K = torch.randn(heads, N, d, generator=g, device=dev).to(torch.bfloat16)
         V = torch.randn(heads, N, d, generator=g, device=dev).to(torch.bfloat16)
@@ -752,6 +815,9 @@ def kernel_case(args):
         if args.case == "dense":
             fn = lambda: tra.tra_dense_attn_entropy(Q, K, V, O_, H)  # noqa: E731
             flops = 4.0 * d * N * N * heads
+        elif args.case == "entropy":
+            fn = lambda: tra.tra_attn_entropy(Q, K, H)  # noqa: E731
+            flops = 2.0 * d * N * N * heads     # QK^T only
         else:
             fn = lambda: tra.tra_block_sparse_attn(Q, K, V, O_, rpd, cid, 128, 128)  # noqa: E731
             flops = 4.0 * d * kept
@@ -794,12 +860,12 @@ def kernel_case(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["dense", "sparse", "mask", "permute"], default=None,
+    ap.add_argument("--case", choices=["dense", "sparse", "entropy", "mask", "permute"], default=None,
                     help="run one kernel on a small case (for profiler captures)")
     ap.add_argument("--reps", type=int, default=3)
-    ap.add_argument("--workload", default="wan14b", choices=sorted(WORKLOADS) + ["sweep", "variants"],
+    ap.add_argument("--workload", default="wan14b", choices=sorted(WORKLOADS) + ["sweep", "variants", "reuse"],
                     help="wan14b (default, the headline step), wan13b, hunyuan, tiny, the "
-                         "density sweep, or the mask variants")
+                         "density sweep, the mask variants, or the reuse policies")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
@@ -817,6 +883,9 @@ def main():
         return
     if args.workload == "variants":
         variants_arm(args)
+        return
+    if args.workload == "reuse":
+        reuse_arm(args)
         return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

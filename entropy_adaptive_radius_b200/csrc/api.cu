@@ -163,6 +163,23 @@ tra_status tra_dense_attn_entropy(const void* Q, const void* K, const void* V, v
   return status_of(launch_attention(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+tra_status tra_attn_entropy(const void* Q, const void* K, float* H, float* lse, int heads, int N,
+                            int d, float scale, tra_stream_t stream) {
+  if (heads < 0 || N < 0) return TRA_ERR_INVALID_ARGUMENT;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return TRA_ERR_INVALID_ARGUMENT;
+  if (d != 64 && d != 128) return TRA_ERR_UNSUPPORTED;
+  if (heads == 0 || N == 0) return TRA_OK;
+  if (heads > 65535 || N > (1 << 24)) return TRA_ERR_UNSUPPORTED;
+  if (!Q || !K || !H || !aligned16(Q) || !aligned16(K)) return TRA_ERR_INVALID_ARGUMENT;
+  const tra_status s = check_device();
+  if (s != TRA_OK) return s;
+  AttnArgs a{};
+  a.Q = Q; a.K = K; a.V = nullptr; a.O = nullptr; a.H = H; a.lse = lse;
+  a.heads = heads; a.N = N; a.d = d; a.scale = scale; a.dense = true; a.entropy_only = true;
+  a.block_q = 128; a.block_k = 128;
+  return status_of(launch_attention(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 tra_status tra_block_sparse_attn(const void* Q, const void* K, const void* V, void* O, float* lse,
                                  const int* row_ptr, const int* col_idx, int heads, int N, int d,
                                  int block_q, int block_k, float scale, tra_stream_t stream) {

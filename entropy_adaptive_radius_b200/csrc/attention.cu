@@ -1167,6 +1167,249 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Entropy-only pass: H and LSE of every query over all N keys, without the
+// PV product or the output (an entropy refresh that needs no dense output).
+//
+// Same split as the two-warpgroup kernel: warpgroup w takes key blocks
+// j = w, w + 2, ...; with no output accumulator each warpgroup has two TMEM
+// score tiles (S_{w,0}, S_{w,1}), so the MMA warp can run two of its QK
+// products ahead.  K has a 4-stage ring.  Per score the softmax does one
+// packed FMA (x = s * scale * log2 e - m), one ex2 and half of a packed add
+// (Z) and of a packed FMA (A): the MUFU unit bounds it, the tensor cores run
+// at half their dense-pass load.  Warps: 0..7 softmax, 8 Q/K producer (and
+// tensor-memory allocation), 9 MMA.
+// ---------------------------------------------------------------------------
+
+constexpr int kEntThreads = 320;  // 10 warps
+constexpr int kEntKWarp = 8;
+constexpr int kEntMmaWarp = 9;
+
+template <int D>
+struct EntCfg {
+  static constexpr int BK = 128;
+  static constexpr int NS = 4;
+  static constexpr int KCH = D / 64;
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BK * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_ST = OFF_K + NS * KV_BYTES;  // merge statistics, 2 x 3 x 128 fp32
+  static constexpr int OFF_BAR = OFF_ST + 2 * 3 * BM * 4;
+  static constexpr int NUM_BARS = 1 + 2 * NS + 8 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + 256;
+  static constexpr int USED = OFF_MISC + 64;
+  static constexpr int SMEM = (USED < 120 * 1024 ? 120 * 1024 : USED) + 1024;
+  static constexpr int TMEM_COLS = 512;  // S_{0,0}, S_{0,1}, S_{1,0}, S_{1,1}
+  static_assert(4 * BK <= TMEM_COLS, "tensor memory");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(NUM_BARS * 8 <= 256, "barrier area");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kEntThreads, 1)
+    entropy_kernel(const __grid_constant__ CUtensorMap tmQ,
+                   const __grid_constant__ CUtensorMap tmK, const Params p) {
+  using C = EntCfg<D>;
+  constexpr int NS = C::NS;
+  constexpr int BK = C::BK;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::OFF_Q;
+  const uint32_t sK = sbase + C::OFF_K;
+  const uint32_t bars = sbase + C::OFF_BAR;
+  const uint32_t bar_q = bars;
+  auto k_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto k_empty = [&](int s) { return bars + 8u * (1 + NS + s); };
+  auto s_full = [&](int t) { return bars + 8u * (1 + 2 * NS + t); };   // t = 2 w + buffer
+  auto s_free = [&](int t) { return bars + 8u * (5 + 2 * NS + t); };
+  const uint32_t drain_bar = bars + 8u * (9 + 2 * NS);
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
+  volatile int* abort = misc + 1;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int qt = blockIdx.x, h = blockIdx.y;
+  const int nblk = p.nkb;
+
+  if (tid == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+    }
+    for (int t = 0; t < 4; ++t) {
+      mbar_init(s_full(t), 1);
+      mbar_init(s_free(t), 128);
+    }
+    mbar_init(drain_bar, 1);
+    fence_barrier_init();
+    misc[1] = 0;
+  }
+  if (warp == kEntKWarp) {
+    tmem_alloc(smem_u32(const_cast<int*>(misc)), C::TMEM_COLS);
+    tmem_relinquish();
+    if (lane == 0) {
+      tma_prefetch_map(&tmQ);
+      tma_prefetch_map(&tmK);
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+
+  if (warp == kEntKWarp) {
+    // ===================================================== Q / K producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * (BM * 128), &tmQ, c * 64, qt * BM, h, bar_q);
+      int issued = 0;
+      for (int j = 0; j < nblk; ++j) {
+        const int s = j % NS;
+        if (!mbar_wait(k_empty(s), ((j / NS) & 1) ^ 1u, abort, p.err, kErrWaitKEmpty)) break;
+        mbar_arrive_expect_tx(k_full(s), C::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sK + s * C::KV_BYTES + c * (BK * 128), &tmK, c * 64, j * BK, h, k_full(s));
+        issued = j + 1;
+      }
+      if (*abort) {
+        drain_wait(bar_q, 0);
+        for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
+          drain_wait(k_full(j % NS), (j / NS) & 1);
+      }
+    }
+  } else if (warp == kEntMmaWarp) {
+    // ===================================================== MMA issuer (QK only, in block order)
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BK, 0, 0);
+      bool ok = mbar_wait(bar_q, 0, abort, p.err, kErrWaitQ);
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int s = j % NS, w = j & 1, i = j >> 1, t = 2 * w + (i & 1), u = i >> 1;
+        ok = mbar_wait(k_full(s), (j / NS) & 1, abort, p.err, kErrWaitKFull) &&
+             mbar_wait(s_free(t), (u & 1) ^ 1u, abort, p.err, kErrWaitSFree);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tS = tmem + t * BK;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t a = smem_desc_sw128(sQ + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              smem_desc_sw128(sK + s * C::KV_BYTES + (k >> 2) * (BK * 128) + (k & 3) * 32, 16, 1024);
+          mma_bf16_ss(tS, a, bd, kIdescQK, k > 0 ? 1u : 0u);
+        }
+        mma_commit(k_empty(s));
+        mma_commit(s_full(t));
+      }
+      if (!ok) {
+        mma_commit(drain_bar);
+        drain_wait(drain_bar, 0);
+      }
+    }
+  } else if (warp < 8) {
+    // ===================================================== softmax statistics (warps 0..7)
+    const int w = warp >> 2;
+    const int row = tid & 127;
+    const uint32_t tl = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int qpos = qt * BM + row;
+    const int nmine = (nblk + 1 - w) >> 1;
+    float m_ref = -INFINITY, Z = 0.f, A = 0.f;
+    bool ok = true;
+    float sv[BK];
+    for (int i = 0; i < nmine; ++i) {
+      const int j = 2 * i + w;
+      const int t = 2 * w + (i & 1), u = i >> 1;
+      ok = mbar_wait(s_full(t), u & 1, abort, p.err, kErrWaitSFull);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < BK / 32; ++c) tmem_ld32f(tmem + tl + t * BK + c * 32, sv + c * 32);
+      tmem_wait_ld();
+      freg_fence<BK>(sv);
+      tc_fence_before();
+      mbar_arrive(s_free(t));
+      const int nvalid = min(BK, p.N - j * BK);  // keys past N (zero rows) are excluded
+      if (nvalid < BK) {
+#pragma unroll
+        for (int c = 0; c < BK; ++c) sv[c] = c < nvalid ? sv[c] : -1e30f;
+      }
+      {
+        float mx[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          mx[q] = fmax3(sv[q], sv[16 + q], sv[32 + q]);
+          mx[q] = fmax3(mx[q], sv[48 + q], sv[64 + q]);
+          mx[q] = fmax3(mx[q], sv[80 + q], sv[96 + q]);
+          mx[q] = fmaxf(mx[q], sv[112 + q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 5; ++q) mx[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
+        const float bmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[15])) *
+                           p.scale_log2;
+        const float m_new = fmaxf(m_ref, bmax);
+        if (m_new > m_ref + kRescaleLog2) {
+          if (m_ref != -INFINITY) {
+            const float alpha = ex2_approx(m_ref - m_new);
+            A = alpha * (A + (m_ref - m_new) * Z);
+            Z *= alpha;
+          }
+          m_ref = m_new;
+        }
+      }
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 nm2 = make_float2(-m_ref, -m_ref);
+      float2 z2[4], a2[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        z2[q] = make_float2(0.f, 0.f);
+        a2[q] = make_float2(0.f, 0.f);
+      }
+#pragma unroll
+      for (int c = 0; c < BK / 2; ++c) {
+        const float2 x = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nm2);
+        const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        z2[c & 3] = __fadd2_rn(z2[c & 3], pr);
+        a2[c & 3] = __ffma2_rn(pr, x, a2[c & 3]);
+      }
+      const float2 zz = __fadd2_rn(__fadd2_rn(z2[0], z2[1]), __fadd2_rn(z2[2], z2[3]));
+      const float2 aa = __fadd2_rn(__fadd2_rn(a2[0], a2[1]), __fadd2_rn(a2[2], a2[3]));
+      Z += zz.x + zz.y;
+      A += aa.x + aa.y;
+    }
+    // ---- merge the two warpgroups' statistics; warpgroup 0 writes H and LSE
+    float* st = reinterpret_cast<float*>(smem + C::OFF_ST);
+    st[(w * 3 + 0) * BM + row] = ok ? m_ref : -INFINITY;
+    st[(w * 3 + 1) * BM + row] = ok ? Z : 0.f;
+    st[(w * 3 + 2) * BM + row] = ok ? A : 0.f;
+    named_barrier_sync(1, 256);
+    if (w == 0 && qpos < p.N) {
+      const float m0 = st[0 * BM + row], Z0 = st[1 * BM + row], A0 = st[2 * BM + row];
+      const float m1 = st[3 * BM + row], Z1 = st[4 * BM + row], A1 = st[5 * BM + row];
+      const float m = fmaxf(m0, m1);
+      const float a0 = (m0 == -INFINITY) ? 0.f : ex2_approx(m0 - m);
+      const float a1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - m);
+      const float Zt = a0 * Z0 + a1 * Z1;
+      float At = 0.f;
+      if (a0 > 0.f) At += a0 * (A0 + (m0 - m) * Z0);
+      if (a1 > 0.f) At += a1 * (A1 + (m1 - m) * Z1);
+      const size_t idx = static_cast<size_t>(h) * p.N + qpos;
+      p.H[idx] = Zt > 0.f ? logf(Zt) - kLn2 * (At / Zt) : NAN;
+      if (p.lse != nullptr) p.lse[idx] = Zt > 0.f ? kLn2 * (m + log2f(Zt)) : -INFINITY;
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == kEntKWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -1216,6 +1459,20 @@ cudaError_t launch_dual(const AttnArgs& a, const Params& prm, cudaStream_t strea
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t launch_entropy(const AttnArgs& a, const Params& prm, cudaStream_t stream) {
+  using C = EntCfg<D>;
+  CUtensorMap mq, mk;
+  if (!make_map(&mq, a.Q, D, a.N, a.heads, BM) || !make_map(&mk, a.K, D, a.N, a.heads, 128))
+    return cudaErrorInvalidValue;
+  auto kern = entropy_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((a.N + BM - 1) / BM, a.heads);
+  kern<<<grid, kEntThreads, C::SMEM, stream>>>(mq, mk, prm);
+  return cudaGetLastError();
+}
+
 template <int D, int BK, bool DENSE>
 cudaError_t launch_cfg(const AttnArgs& a, const Params& prm, cudaStream_t stream) {
   using C = Cfg<D, BK>;
@@ -1252,6 +1509,8 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
   // Query and key blocks of 64 or 128 tokens (and the dense pass) use the
   // two-warpgroup kernel; 16-token blocks use the single-warpgroup kernel,
   // which merges the lists of up to eight query blocks per CTA.
+  if (a.entropy_only) return a.d == 128 ? launch_entropy<128>(a, prm, stream)
+                                          : launch_entropy<64>(a, prm, stream);
   if (a.dense) {
     if (a.d == 128) return launch_dual<128, 128, true>(a, prm, stream);
     return launch_dual<64, 128, true>(a, prm, stream);

@@ -63,6 +63,7 @@ struct AttnArgs {
   int block_q, block_k;  // sparse only; dense uses 128-key tiles
   float scale;
   bool dense;
+  bool entropy_only;  // H (and LSE) over all keys, no output (V and O unused)
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream);
 

@@ -1,0 +1,118 @@
+"""One Token Radius Attention layer across the denoising steps of a video
+diffusion model (Token Radius Attention summary, §2 "TRA pipeline": entropy
+from a dense warm-up phase, budget -> radius -> block mask, and cross-step
+reuse of the entropy by the later sparse steps).
+
+`TraLayer` owns the device buffers of one layer: the tile-major copies of
+Q, K, V and O, the entropy, radii, decay table, the CSR block mask and the
+mask's scratch space.  Its `forward` runs one step through the C ABI; which
+kind of step it is follows the `ReusePolicy`:
+
+  * the first `warmup` steps are dense: dense attention with entropy, then
+    radius and mask from that entropy;
+  * every later step is sparse: block-sparse attention over the current mask;
+  * with `refresh_every = k > 0`, every k-th step after the warm-up also
+    refreshes the entropy from its own Q and K and rebuilds the mask for the
+    steps that follow: `refresh = "entropy"` keeps the sparse output and adds
+    an entropy-only pass (no PV product); `refresh = "dense"` makes the step a
+    dense one.
+
+This module only sequences calls and holds buffers; every step of the method
+runs in the CUDA kernels behind `tra`.
+"""
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+from . import tra
+
+
+@dataclass(frozen=True)
+class ReusePolicy:
+    warmup: int = 1
+    refresh_every: int = 0
+    refresh: str = "entropy"  # "entropy" (entropy-only pass) or "dense"
+
+    def __post_init__(self):
+        if self.warmup < 1:
+            raise ValueError("the first step must be dense: warmup >= 1")
+        if self.refresh_every < 0:
+            raise ValueError("refresh_every >= 0")
+        if self.refresh not in ("entropy", "dense"):
+            raise ValueError("refresh is 'entropy' or 'dense'")
+
+    def kind(self, step: int) -> str:
+        """"dense", "sparse" or "sparse+entropy" for step index `step`."""
+        if step < self.warmup:
+            return "dense"
+        k = step - self.warmup + 1  # 1-based index in the sparse phase
+        if self.refresh_every and k % self.refresh_every == 0:
+            return "dense" if self.refresh == "dense" else "sparse+entropy"
+        return "sparse"
+
+
+class TraLayer:
+    """Buffers and step sequencing of one attention layer on one GPU."""
+
+    def __init__(self, grid: Sequence[int], heads: int, d: int, *, tau: float, gamma: float,
+                 tile=(1, 4, 4), block_q: int = 128, block_k: int = 128, vote: int = 1,
+                 policy: ReusePolicy = ReusePolicy(), device="cuda"):
+        self.grid = tuple(int(v) for v in grid)
+        F, H, W = self.grid
+        self.N = F * H * W
+        self.heads, self.d = heads, d
+        self.tile = tuple(tile)
+        self.block_q, self.block_k = block_q, block_k
+        self.tau, self.gamma, self.vote = float(tau), float(gamma), int(vote)
+        self.policy = policy
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.Qtm, self.Ktm, self.Vtm, self.Otm = (torch.empty(heads, self.N, d, **bf) for _ in range(4))
+        self.H = torch.empty(heads, self.N, dtype=torch.float32, device=device)
+        self.r = torch.empty_like(self.H)
+        self.phi = torch.empty(F, dtype=torch.float32, device=device)
+        self.nqb = -(-self.N // block_q)
+        self.nkb = -(-self.N // block_k)
+        self.row_ptr = torch.empty(heads * (self.nqb + 1), dtype=torch.int32, device=device)
+        self.col_idx = torch.empty(max(1, heads * self.nqb * self.nkb), dtype=torch.int32,
+                                   device=device)
+        self.nnz = torch.zeros(1, dtype=torch.int32, device=device)
+        self.ws = tra.workspace_tensor(
+            tra.tra_mask_workspace_size(heads, self.grid, block_q, block_k, self.tile), device)
+        self.step_index = 0
+
+    def reset(self):
+        """Start a new denoising run (the next step is a warm-up step again)."""
+        self.step_index = 0
+
+    def _rebuild_mask(self):
+        tra.tra_budget_radius(self.H, self.r, self.grid, self.tau, self.gamma, self.tile,
+                              phi_out=self.phi)
+        tra.tra_build_block_mask(self.r, self.phi, self.grid, self.block_q, self.block_k,
+                                 self.vote, self.row_ptr, self.col_idx, self.nnz, self.ws,
+                                 self.tile)
+
+    def forward(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                O: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """One denoising step.  Q, K, V: [heads, N, d] in the original (t, y, x)
+        token order, bf16 (or fp32, rounded to bf16 by the permute).  Returns
+        O [heads, N, d] bf16 in the original order."""
+        kind = self.policy.kind(self.step_index)
+        if O is None:
+            O = torch.empty(self.heads, self.N, self.d, dtype=torch.bfloat16, device=Q.device)
+        for X, Y in ((Q, self.Qtm), (K, self.Ktm), (V, self.Vtm)):
+            tra.tra_tile_major_permute(X, Y, self.grid, self.tile)
+        if kind == "dense":
+            tra.tra_dense_attn_entropy(self.Qtm, self.Ktm, self.Vtm, self.Otm, self.H)
+            self._rebuild_mask()
+        else:
+            tra.tra_block_sparse_attn(self.Qtm, self.Ktm, self.Vtm, self.Otm, self.row_ptr,
+                                      self.col_idx, self.block_q, self.block_k)
+            if kind == "sparse+entropy":
+                tra.tra_attn_entropy(self.Qtm, self.Ktm, self.H)
+                self._rebuild_mask()
+        tra.tra_inverse_permute(self.Otm, O, self.grid, self.tile)
+        self.step_index += 1
+        return O
+
+    __call__ = forward

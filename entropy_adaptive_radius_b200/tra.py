@@ -52,6 +52,7 @@ _PROTOS = {
     "tra_inverse_permute": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, Grid, Tile, _vp]),
     "tra_dense_attn_entropy": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                                         _c_float, _vp]),
+    "tra_attn_entropy": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_float, _vp]),
     "tra_budget_radius": (_c_int, [_vp, _vp, _vp, _c_int, Grid, Tile, _c_float, _c_float, _vp]),
     "tra_budget_radius_ex": (_c_int, [_vp, _vp, _vp, _c_int, Grid, Tile, _c_float, _c_float,
                                       _c_int, _c_int, _vp]),
@@ -155,6 +156,17 @@ def tra_dense_attn_entropy(Q, K, V, O, H, lse=None, scale=None, stream=None):
     _check("tra_dense_attn_entropy", lib().tra_dense_attn_entropy(
         _p(Q), _p(K), _p(V), _p(O), _p(H), _p(lse), heads, N, d, scale, _stream(stream)))
     return O, H
+
+
+def tra_attn_entropy(Q, K, H, lse=None, scale=None, stream=None):
+    """Entropy H (and optionally LSE) of every query of Q, K [heads, N, d] bf16
+    over all keys, without the PV product or an output."""
+    _contig(Q, K, H, lse)
+    heads, N, d = Q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    _check("tra_attn_entropy", lib().tra_attn_entropy(
+        _p(Q), _p(K), _p(H), _p(lse), heads, N, d, scale, _stream(stream)))
+    return H
 
 
 def tra_budget_radius(H, r, grid, tau, gamma, tile=(1, 4, 4), phi_out=None, stream=None):

@@ -116,6 +116,19 @@ tra_status tra_dense_attn_entropy(const void* Q, const void* K, const void* V, v
                                   tra_stream_t stream);
 
 /*
+ * Entropy-only pass: the H_i (and lse_i) of tra_dense_attn_entropy without
+ * the PV product and without writing an output.  For refreshing the entropy
+ * (and so the mask) at a step whose output comes from the block-sparse call
+ * (§2 "TRA pipeline", cross-step reuse: the entropy pattern is stable across
+ * denoising steps, so it is recomputed only now and then).
+ *   Q, K  [heads, N, d] bf16, 16-byte aligned; read only.
+ *   H     [heads, N] fp32; written.    lse  [heads, N] fp32 or NULL.
+ *   d 64 or 128; scale > 0 and finite; N 1 .. 2^24.
+ */
+tra_status tra_attn_entropy(const void* Q, const void* K, float* H, float* lse, int heads, int N,
+                            int d, float scale, tra_stream_t stream);
+
+/*
  * Entropy -> budget -> radius (§2 Insight I: B_i = tau * exp(H_i) / N;
  * Insight II and pipeline step 2: budget -> query-specific base radius,
  * per-frame radius r_i * phi(|dt|), phi(delta) = exp(-gamma * delta)).

@@ -55,6 +55,15 @@ Video Generation", abstract), all through the same token mask and votes:
       the temporal distance doubles the window's area (length) halves, so every
       band of temporal distances holds the same number of keys and a query's
       support grows with log F (the O(n log n) cost the Radial page states).
+
+Cross-step reuse (§2 "TRA pipeline": the entropy is computed in the dense
+warm-up phase and reused by the later sparse steps):
+  R15 the first `warmup` steps are dense (output and entropy); every later
+      step is sparse with the mask of the last entropy refresh; with
+      refresh_every = k > 0, every k-th sparse-phase step also refreshes the
+      entropy from its own Q and K, either as a dense step ("dense": dense
+      output) or after its sparse output ("entropy": an entropy-only pass);
+      the new mask serves the steps after it.
 """
 import math
 
@@ -371,3 +380,57 @@ def sparse_attention_rows(Qh, Kh, Vh, mask_h, Bq, Bk, scale, rows):
 
 def kept_fraction(mask):
     return float(np.mean(mask))
+
+
+# ---------------------------------------------------------------------------
+# cross-step reuse  (§2 "TRA pipeline", cross-step reuse; reading R15)
+# ---------------------------------------------------------------------------
+
+
+def reuse_plan(steps, warmup, refresh_every, refresh):
+    """Kind of each denoising step: "dense" (dense output, entropy and mask
+    from this step), "sparse" (sparse output over the current mask) or
+    "sparse+entropy" (sparse output, then entropy and mask from this step)."""
+    plan = []
+    for k in range(steps):
+        if k < warmup:
+            plan.append("dense")
+        elif refresh_every > 0 and (k - warmup + 1) % refresh_every == 0:
+            plan.append("dense" if refresh == "dense" else "sparse+entropy")
+        else:
+            plan.append("sparse")
+    return plan
+
+
+def mask_from_entropy(H, coords_tm, tau, gamma, F, Bq, Bk, vote):
+    """Kept-block mask [heads, nqb, nkb] of entropies H [heads, N]: radius by
+    R4 rounded to fp32, phi rounded to fp32, brute-force block votes."""
+    N = coords_tm.shape[0]
+    phi32 = phi(np.arange(F), gamma).astype(np.float32)
+    masks = []
+    for h in range(H.shape[0]):
+        r32 = radius(H[h], coords_tm[:, 2], tau, gamma, F, N).astype(np.float32)
+        masks.append(block_mask(r32, phi32, coords_tm, Bq, Bk, vote))
+    return np.stack(masks)
+
+
+def reuse_run(steps_qkv, coords_tm, F, tau, gamma, Bq, Bk, vote, plan, scale):
+    """Outputs of a denoising schedule.  steps_qkv: per step (Q, K, V) [heads,
+    N, d] in tile-major order.  Returns (outputs, masks used, entropies of
+    the refresh steps)."""
+    outputs, used, refreshed = [], [], {}
+    mask = None
+    for k, ((Q, K, V), kind) in enumerate(zip(steps_qkv, plan)):
+        if kind == "dense":
+            O, H, _ = dense_attention_entropy(Q, K, V, scale)
+            used.append(None)
+        else:
+            O, _ = sparse_attention(Q, K, V, mask, Bq, Bk, scale)
+            used.append(mask)
+            if kind == "sparse+entropy":
+                _, H, _ = dense_attention_entropy(Q, K, V, scale)
+        if kind != "sparse":
+            refreshed[k] = H
+            mask = mask_from_entropy(H, coords_tm, tau, gamma, F, Bq, Bk, vote)
+        outputs.append(O)
+    return outputs, used, refreshed
