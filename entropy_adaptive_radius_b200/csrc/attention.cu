@@ -596,8 +596,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 // exactly:
 //   m = max(m_0, m_1),  a_w = 2^(m_w - m),  Z = a_0 Z_0 + a_1 Z_1,
 //   A = sum_w a_w (A_w + (m_w - m) Z_w),      O = (a_0 O_0 + a_1 O_1) / Z.
-// Warps: 0..7 softmax, 8 Q/K producer (and tensor-memory allocation), 9 MMA,
-// 10 V producer.
+// Warps: 0..7 softmax, 8 Q/K producer (and tensor-memory allocation), 9 QK
+// issuer, 10 V producer, 11 PV issuer.  QK and PV are issued by two threads,
+// each in block order and each sleeping in its own barrier waits, so neither
+// stream holds back the other and no warp spins on the softmax warps' issue
+// slots.  The third warpgroup (warps 8..11) hands registers to the two
+// softmax warpgroups (setmaxnreg): 168 per thread at launch, 56 for the
+// producers and issuers, 224 for the softmax.
 //
 // Key blocks of 64 tokens are taken two at a time: a "super-block" of 128
 // keys is the next two entries of the CTA's key-block list, each loaded into
@@ -608,10 +613,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 // itself, in the same order.
 // ---------------------------------------------------------------------------
 
-constexpr int kDualThreads = 352;  // 11 warps
+constexpr int kDualThreads = 384;  // 12 warps
 constexpr int kDualKWarp = 8;
-constexpr int kDualMmaWarp = 9;
+constexpr int kDualQKWarp = 9;
 constexpr int kDualVWarp = 10;
+constexpr int kDualPVWarp = 11;
+// Register split.  The CTA is launched with kDualLaunchRegs per thread (the
+// host refuses to launch a build that allocated anything else); the split
+// hands exactly that pool out again, so setmaxnreg.inc never waits.
+constexpr int kDualLaunchRegs = 168;
+constexpr int kDualRegsOther = 56;
+constexpr int kDualRegsSoftmax = 224;
+static_assert(256 * kDualRegsSoftmax + 128 * kDualRegsOther == kDualThreads * kDualLaunchRegs,
+              "register split must equal the launch pool");
+static_assert(2 * kDualRegsSoftmax * 32 + kDualRegsOther * 32 <= 16384,
+              "per-scheduler register file: two softmax warps and one other warp");
 
 template <int D>
 struct DualCfg {
@@ -626,7 +642,7 @@ struct DualCfg {
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
   static constexpr int OFF_P = OFF_V + NS * KV_BYTES;  // P_0, P_1
   static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-  static constexpr int NUM_BARS = 1 + 4 * NS + 8 + 1;
+  static constexpr int NUM_BARS = 1 + 4 * NS + 8 + 2;
   static constexpr int OFF_MISC = OFF_BAR + 256;
   static constexpr int USED = OFF_MISC + 64;
   static constexpr int SMEM = (USED < 120 * 1024 ? 120 * 1024 : USED) + 1024;
@@ -699,7 +715,8 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   auto s_free = [&](int w) { return bars + 8u * (3 + 4 * NS + w); };
   auto p_full = [&](int w) { return bars + 8u * (5 + 4 * NS + w); };
   auto pv_done = [&](int w) { return bars + 8u * (7 + 4 * NS + w); };
-  const uint32_t drain_bar = bars + 8u * (9 + 4 * NS);
+  const uint32_t drain_qk = bars + 8u * (9 + 4 * NS);
+  const uint32_t drain_pv = bars + 8u * (10 + 4 * NS);
   volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   volatile int* abort = misc + 1;
 
@@ -721,7 +738,8 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       mbar_init(p_full(w), 128);
       mbar_init(pv_done(w), 1);
     }
-    mbar_init(drain_bar, 1);
+    mbar_init(drain_qk, 1);
+    mbar_init(drain_pv, 1);
     fence_barrier_init();
     misc[1] = 0;
     // misc[2] super-blocks, misc[3..6] start / length of CSR rows a and b
@@ -778,6 +796,9 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     }
   };
 
+  if (warp >= 8) {
+  // warpgroup 2 gives registers back (all four warps, same instruction)
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDualRegsOther));
   if (warp == kDualKWarp) {
     // ===================================================== Q / K producer
     if (lane == 0) {
@@ -836,21 +857,17 @@ __global__ void __launch_bounds__(kDualThreads, 1)
           drain_wait(v_full(j % NS), (j / NS) & 1);
       }
     }
-  } else if (warp == kDualMmaWarp) {
-    // ===================================================== MMA issuer
+  } else if (warp == kDualQKWarp) {
+    // ===================================================== QK issuer (block order)
+    // QK_j needs K_j and the release of S_{j mod 2} by block j - 2's softmax.
     if (lane == 0) {
       constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BK, 0, 0);
-      constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, D, 0, 1);
-      auto qk_ready = [&](int j) -> bool {
+      bool ok = mbar_wait(bar_q, 0, abort, p.err, kErrWaitQ);
+      for (int j = 0; ok && j < nblk; ++j) {
         const int s = j % NS, w = j & 1, i = j >> 1;
-        return mbar_test(k_full(s), (j / NS) & 1) && mbar_test(s_free(w), (i & 1) ^ 1u);
-      };
-      auto pv_ready = [&](int j) -> bool {
-        const int s = j % NS, w = j & 1, i = j >> 1;
-        return mbar_test(p_full(w), i & 1) && mbar_test(v_full(s), (j / NS) & 1);
-      };
-      auto issue_qk = [&](int j) {
-        const int s = j % NS, w = j & 1;
+        ok = mbar_wait(k_full(s), (j / NS) & 1, abort, p.err, kErrWaitKFull) &&
+             mbar_wait(s_free(w), (i & 1) ^ 1u, abort, p.err, kErrWaitSFree);
+        if (!ok) break;
         tc_fence_after();
         const uint32_t tS = tmem + w * BK;
 #pragma unroll
@@ -862,9 +879,23 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         }
         mma_commit(k_empty(s));
         mma_commit(s_full(w));
-      };
-      auto issue_pv = [&](int j) {
+      }
+      if (!ok) {
+        mma_commit(drain_qk);
+        drain_wait(drain_qk, 0);
+      }
+    }
+  } else if (warp == kDualPVWarp) {
+    // ===================================================== PV issuer (block order)
+    // PV_j needs P_j from warpgroup j mod 2 and V_j.
+    if (lane == 0) {
+      constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, D, 0, 1);
+      bool ok = true;
+      for (int j = 0; ok && j < nblk; ++j) {
         const int s = j % NS, w = j & 1, i = j >> 1;
+        ok = mbar_wait(p_full(w), i & 1, abort, p.err, kErrWaitPFull) &&
+             mbar_wait(v_full(s), (j / NS) & 1, abort, p.err, kErrWaitVFull);
+        if (!ok) break;
         tc_fence_after();
         const uint32_t tO = tmem + 2 * BK + w * D;
         const uint32_t pw = sP + w * C::P_BYTES;
@@ -876,47 +907,17 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         }
         mma_commit(v_empty(s));
         mma_commit(pv_done(w));
-      };
-      // Issue QK and PV in whatever order their inputs become ready, so that
-      // one warpgroup's softmax never holds back the other's next score tile.
-      // QK_j needs K_j and the release of S_{j mod 2} (block j-2); PV_j needs
-      // P_j and V_j.  Both streams stay in block order.
-      bool ok = mbar_wait(bar_q, 0, abort, p.err, kErrWaitQ);
-      int nq = 0, np = 0;
-      unsigned long long t_idle = 0;
-      int idle = 0;
-      while (ok && np < nblk) {
-        bool did = false;
-        if (nq < nblk && qk_ready(nq)) {
-          issue_qk(nq++);
-          did = true;
-        }
-        if (np < nq && pv_ready(np)) {
-          issue_pv(np++);
-          did = true;
-        }
-        if (did) {
-          idle = 0;
-        } else if (++idle == 1) {
-          t_idle = global_timer_ns();
-        } else if ((idle & 255) == 0) {
-          // nothing ready for a while: give up after the usual time limit
-          if (*abort) {
-            ok = false;
-          } else if (global_timer_ns() - t_idle > kWaitTimeoutNs) {
-            *abort = 1;
-            if (p.err) atomicCAS(p.err, 0, kErrWaitPFull);
-            ok = false;
-          }
-        }
       }
       if (!ok) {
-        mma_commit(drain_bar);
-        drain_wait(drain_bar, 0);
+        mma_commit(drain_pv);
+        drain_wait(drain_pv, 0);
       }
     }
-  } else if (warp < 8) {
+  }
+  } else {
     // ===================================================== softmax warpgroups (warps 0..7)
+    // take the registers warpgroup 2 gave back (waits until it has)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kDualRegsSoftmax));
     const int w = warp >> 2;                  // warpgroup 0 or 1
     const int row = tid & 127;                // query row = TMEM lane
     const uint32_t tl = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -940,25 +941,36 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     ListWalker wk = make_walker();
     int dn = 0, sb_done = 0;
     const uint32_t my_bit = (p.G == 2) ? (1u << (row >> 6)) : 1u;
+    // One query block per CTA and one list entry per super-block (128-row
+    // query blocks, 128-key blocks, and the dense pass): every row keeps every
+    // entry, so entry j is simply the j-th list element (one load, no walk)
+    const bool direct = (E == 1) && (DENSE || p.G == 1);
+    const int* my_list = p.col_idx + misc[3];
     for (int i = 0; i < nmine; ++i) {
       const int j = 2 * i + w;
-      // entries of super-block j (skipping the other warpgroup's)
+      // valid keys of each entry of super-block j for this row
       int nv[E];
-      for (; sb_done < j; ++sb_done) {
+      if (direct) {
+        const int kb = DENSE ? j : __ldg(my_list + j);
+        nv[0] = (kb >= 0 && kb < p.nkb) ? min(BKS, p.N - kb * BKS) : 0;
+      } else {
+        // walk the merged list, skipping the other warpgroup's super-blocks
+        for (; sb_done < j; ++sb_done) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            uint32_t mem;
+            next_entry(wk, dn, mem);
+          }
+        }
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           uint32_t mem;
-          next_entry(wk, dn, mem);
+          const int kb = next_entry(wk, dn, mem);
+          const bool keep = kb >= 0 && kb < p.nkb && (mem & my_bit) != 0u;
+          nv[e] = keep ? min(BKS, p.N - kb * BKS) : 0;
         }
+        ++sb_done;
       }
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        uint32_t mem;
-        const int kb = next_entry(wk, dn, mem);
-        const bool keep = kb >= 0 && kb < p.nkb && (mem & my_bit) != 0u;
-        nv[e] = keep ? min(BKS, p.N - kb * BKS) : 0;
-      }
-      ++sb_done;
       ok = mbar_wait(s_full(w), i & 1, abort, p.err, kErrWaitSFull);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -1447,11 +1459,18 @@ bool make_map(CUtensorMap* map, const void* base, int d, int N, int heads, int r
 template <int D, int BKS, bool DENSE>
 cudaError_t launch_dual(const AttnArgs& a, const Params& prm, cudaStream_t stream) {
   using C = DualCfg<D>;
+  auto kern = attn_dual_kernel<D, BKS, DENSE>;
+  // The kernel's register split assumes exactly kDualLaunchRegs per thread at
+  // launch; with any other allocation setmaxnreg.inc could wait forever.
+  static const int launch_regs = [kern] {
+    cudaFuncAttributes fa{};
+    return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1;
+  }();
+  if (launch_regs != kDualLaunchRegs) return cudaErrorInvalidDeviceFunction;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, a.Q, D, a.N, a.heads, BM) || !make_map(&mk, a.K, D, a.N, a.heads, BKS) ||
       !make_map(&mv, a.V, D, a.N, a.heads, BKS))
     return cudaErrorInvalidValue;
-  auto kern = attn_dual_kernel<D, BKS, DENSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const dim3 grid((a.N + BM - 1) / BM, a.heads);
