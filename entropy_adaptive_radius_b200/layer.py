@@ -17,6 +17,12 @@ kind of step it is follows the `ReusePolicy`:
     an entropy-only pass (no PV product); `refresh = "dense"` makes the step a
     dense one.
 
+With `layout="tile_major"` the layer takes and returns tensors that are
+already in tile-major order and runs no permutation: a model that keeps the
+tokens of a whole transformer block in tile-major order permutes once on the
+way in and once on the way out (`to_tile_major` / `from_tile_major`) instead
+of around every attention call.
+
 This module only sequences calls and holds buffers; every step of the method
 runs in the CUDA kernels behind `tra`.
 """
@@ -57,7 +63,10 @@ class TraLayer:
 
     def __init__(self, grid: Sequence[int], heads: int, d: int, *, tau: float, gamma: float,
                  tile=(1, 4, 4), block_q: int = 128, block_k: int = 128, vote: int = 1,
-                 policy: ReusePolicy = ReusePolicy(), device="cuda"):
+                 policy: ReusePolicy = ReusePolicy(), layout: str = "original", device="cuda"):
+        if layout not in ("original", "tile_major"):
+            raise ValueError("layout is 'original' or 'tile_major'")
+        self.layout = layout
         self.grid = tuple(int(v) for v in grid)
         F, H, W = self.grid
         self.N = F * H * W
@@ -67,7 +76,10 @@ class TraLayer:
         self.tau, self.gamma, self.vote = float(tau), float(gamma), int(vote)
         self.policy = policy
         bf = dict(dtype=torch.bfloat16, device=device)
-        self.Qtm, self.Ktm, self.Vtm, self.Otm = (torch.empty(heads, self.N, d, **bf) for _ in range(4))
+        # tile-major copies of Q, K, V, O (the resident layout needs none)
+        n_buf = 4 if layout == "original" else 0
+        self.Qtm, self.Ktm, self.Vtm, self.Otm = (
+            [torch.empty(heads, self.N, d, **bf) for _ in range(n_buf)] or [None] * 4)
         self.H = torch.empty(heads, self.N, dtype=torch.float32, device=device)
         self.r = torch.empty_like(self.H)
         self.phi = torch.empty(F, dtype=torch.float32, device=device)
@@ -92,26 +104,44 @@ class TraLayer:
                                  self.vote, self.row_ptr, self.col_idx, self.nnz, self.ws,
                                  self.tile)
 
+    def to_tile_major(self, X: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """[heads, N, d] from the original token order to tile-major order (bf16)."""
+        if out is None:
+            out = torch.empty(X.shape, dtype=torch.bfloat16, device=X.device)
+        return tra.tra_tile_major_permute(X, out, self.grid, self.tile)
+
+    def from_tile_major(self, X_tm: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """[heads, N, d] from tile-major order back to the original order."""
+        if out is None:
+            out = torch.empty_like(X_tm)
+        return tra.tra_inverse_permute(X_tm, out, self.grid, self.tile)
+
     def forward(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                 O: Optional[torch.Tensor] = None) -> torch.Tensor:
-        """One denoising step.  Q, K, V: [heads, N, d] in the original (t, y, x)
-        token order, bf16 (or fp32, rounded to bf16 by the permute).  Returns
-        O [heads, N, d] bf16 in the original order."""
+        """One denoising step.  Q, K, V: [heads, N, d], bf16 (or fp32 in the
+        original layout, rounded to bf16 by the permute), in the original
+        (t, y, x) token order, or in tile-major order with layout="tile_major".
+        Returns O [heads, N, d] bf16 in the same order as the inputs."""
         kind = self.policy.kind(self.step_index)
         if O is None:
             O = torch.empty(self.heads, self.N, self.d, dtype=torch.bfloat16, device=Q.device)
-        for X, Y in ((Q, self.Qtm), (K, self.Ktm), (V, self.Vtm)):
-            tra.tra_tile_major_permute(X, Y, self.grid, self.tile)
+        if self.layout == "original":
+            for X, Y in ((Q, self.Qtm), (K, self.Ktm), (V, self.Vtm)):
+                tra.tra_tile_major_permute(X, Y, self.grid, self.tile)
+            q, k, v, o = self.Qtm, self.Ktm, self.Vtm, self.Otm
+        else:
+            q, k, v, o = Q, K, V, O
         if kind == "dense":
-            tra.tra_dense_attn_entropy(self.Qtm, self.Ktm, self.Vtm, self.Otm, self.H)
+            tra.tra_dense_attn_entropy(q, k, v, o, self.H)
             self._rebuild_mask()
         else:
-            tra.tra_block_sparse_attn(self.Qtm, self.Ktm, self.Vtm, self.Otm, self.row_ptr,
-                                      self.col_idx, self.block_q, self.block_k)
+            tra.tra_block_sparse_attn(q, k, v, o, self.row_ptr, self.col_idx, self.block_q,
+                                      self.block_k)
             if kind == "sparse+entropy":
-                tra.tra_attn_entropy(self.Qtm, self.Ktm, self.H)
+                tra.tra_attn_entropy(q, k, self.H)
                 self._rebuild_mask()
-        tra.tra_inverse_permute(self.Otm, O, self.grid, self.tile)
+        if self.layout == "original":
+            tra.tra_inverse_permute(self.Otm, O, self.grid, self.tile)
         self.step_index += 1
         return O
 

@@ -114,3 +114,25 @@ def test_reuse_loop_matches_oracle_schedule(refresh):
     ms = [O.mask_from_entropy(refreshed[k], c, tau, gamma32, F, BQ, BK, 1) for k in refresh_steps]
     assert any(not np.array_equal(ms[0], m) for m in ms[1:])
     assert all(0.0 < m.mean() < 1.0 for m in ms)
+
+
+def test_tile_major_resident_layer_matches_original_layout():
+    """layout="tile_major" runs the same kernels on already-permuted tensors:
+    its outputs, permuted back, equal the original-layout layer's bit for bit,
+    step by step, and so do the masks."""
+    need_gpu()
+    steps = make_steps(seed=8)
+    policy = ReusePolicy(warmup=1, refresh_every=2, refresh="entropy")
+    kw = dict(tau=0.1, gamma=GAMMA, tile=TILE, block_q=BQ, block_k=BK, policy=policy)
+    a = TraLayer((F, HH, WW), HEADS, D, **kw)
+    b = TraLayer((F, HH, WW), HEADS, D, layout="tile_major", **kw)
+    for Q, K, V in steps:
+        Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+        Oa = a(Qd, Kd, Vd)
+        Ob_tm = b(b.to_tile_major(Qd), b.to_tile_major(Kd), b.to_tile_major(Vd))
+        assert torch.equal(b.from_tile_major(Ob_tm), Oa)
+        assert int(a.nnz.item()) == int(b.nnz.item())
+        assert torch.equal(a.row_ptr, b.row_ptr)
+    assert tra.tra_get_device_error() == 0
+    with pytest.raises(ValueError):
+        TraLayer((F, HH, WW), HEADS, D, layout="diagonal", **kw)
