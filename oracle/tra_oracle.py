@@ -56,6 +56,15 @@ Video Generation", abstract), all through the same token mask and votes:
       band of temporal distances holds the same number of keys and a query's
       support grows with log F (the O(n log n) cost the Radial page states).
 
+FP8 scores (the last "next" row: same mask, QK^T on FP8 tensor cores):
+  R16 Q and K are quantized per (head, block of rows) to OCP FP8 E4M3: the
+      block's scale is fl32(amax / 448) (1 for an all-zero block) and each
+      element becomes the nearest E4M3 value (ties to even, saturating at
+      448) to fl32(x / scale); scores are scale_q * scale_k * (q8 . k8) times
+      the softmax scale, and everything after the scores is unchanged.  The
+      pages say nothing about precision; this is the plainest per-block
+      scaled FP8 reading.
+
 Cross-step reuse (§2 "TRA pipeline": the entropy is computed in the dense
 warm-up phase and reused by the later sparse steps):
   R15 the first `warmup` steps are dense (output and entropy); every later
@@ -434,3 +443,66 @@ def reuse_run(steps_qkv, coords_tm, F, tau, gamma, Bq, Bk, vote, plan, scale):
             mask = mask_from_entropy(H, coords_tm, tau, gamma, F, Bq, Bk, vote)
         outputs.append(O)
     return outputs, used, refreshed
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) scores  (reading R16)
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def round_e4m3(x):
+    """Nearest OCP FP8 E4M3 value (1 sign bit, 4 exponent bits with bias 7, 3
+    mantissa bits, no infinities, largest finite 448), ties to even; finite
+    values beyond +-448 saturate.  The rounding itself is torch's float8_e4m3fn
+    conversion (a library primitive, pinned to the format in the tests)."""
+    import torch
+    x = np.clip(np.asarray(x, np.float32), -E4M3_MAX, E4M3_MAX)
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.float8_e4m3fn).to(
+        torch.float32).numpy().astype(np.float64)
+
+
+def quantize_e4m3_blocks(X, block):
+    """Per head and per block of `block` consecutive rows of X [heads, N, d]:
+    scale = fl32(amax / 448) (1 when the block is all zero) and codes =
+    E4M3(fl32(x / scale)).  Returns (codes [heads, N, d] as float64,
+    scales [heads, nblocks] float32)."""
+    X32 = np.asarray(X, np.float32)
+    heads, N, _ = X32.shape
+    nb = -(-N // block)
+    codes = np.empty(X32.shape, np.float64)
+    scales = np.empty((heads, nb), np.float32)
+    for h in range(heads):
+        for b in range(nb):
+            blk = X32[h, b * block:(b + 1) * block]
+            amax = np.float32(np.max(np.abs(blk))) if blk.size else np.float32(0)
+            sc = np.float32(amax / np.float32(E4M3_MAX)) if amax > 0 else np.float32(1.0)
+            scales[h, b] = sc
+            codes[h, b * block:(b + 1) * block] = round_e4m3((blk / sc).astype(np.float32))
+    return codes, scales
+
+
+def sparse_attention_fp8qk(Q8, qs, K8, ks, V, mask, Bq, Bk, scale, rows=None, head=None):
+    """Exact softmax over the kept blocks with scores
+    s_ij = scale * qs[i // Bq] * ks[j // Bk] * (q8_i . k8_j).  Q8, K8: E4M3
+    codes [heads, N, d] (float64), qs / ks: per-block scales; V as for
+    sparse_attention.  With `head` and `rows`, only those rows of that head."""
+    heads = range(Q8.shape[0]) if head is None else [head]
+    outs, lses = [], []
+    for h in heads:
+        N = K8.shape[1]
+        r = np.arange(Q8.shape[1]) if rows is None else np.asarray(rows)
+        s = (Q8[h][r] @ K8[h].T) * (np.float64(scale) * qs[h][r // Bq].astype(np.float64)[:, None]
+                                      * ks[h][np.arange(N) // Bk].astype(np.float64)[None, :])
+        km = key_mask_from_blocks(mask[h], r, Bq, Bk, N)
+        s = np.where(km, s, -np.inf)
+        m = np.max(s, axis=1, keepdims=True)
+        ok = np.isfinite(m)
+        e = np.where(km & ok, np.exp(s - np.where(ok, m, 0.0)), 0.0)
+        Z = e.sum(axis=1, keepdims=True)
+        O = np.where(Z > 0, (e @ np.asarray(V[h], np.float64)) / np.where(Z > 0, Z, 1.0), 0.0)
+        L = np.where(Z[:, 0] > 0, np.log(np.where(Z[:, 0] > 0, Z[:, 0], 1.0)) + np.where(ok[:, 0], m[:, 0], 0.0), -np.inf)
+        outs.append(O)
+        lses.append(L)
+    return (np.stack(outs), np.stack(lses)) if head is None else (outs[0], lses[0])
