@@ -852,8 +852,9 @@ def reference_arm(args, rank, world):
 
 def kernel_case(args):
     """Small single-kernel cases for profiler captures (inputs > L2, < 1 GB):
-    dense / sparse / entropy (entropy only, no PV): 40 heads x 16384 tokens x
-    d=128 bf16 (168 MB per tensor);
+    dense / sparse / entropy (entropy only, no PV) / sparse_fp8 (E4M3 Q, K) /
+    quant (E4M3 quantization of Q): 40 heads x 16384 tokens x d=128 bf16
+    (168 MB per tensor);
     mask: the 21x45x80 grid, 40 heads, radii from entropies near ln N;
     permute: one 21x45x80 x 40-head x 128 bf16 tensor.  Runs the kernel
     `--reps` times and prints the mean CUDA-event time per launch."""
@@ -863,7 +864,7 @@ def kernel_case(args):
     g = torch.Generator(device=dev).manual_seed(0)
     heads, N, d = 40, 16384, 128
     reps = args.reps
-    if args.case in ("dense", "sparse", "entropy"):
+    if args.case in ("dense", "sparse", "sparse_fp8", "quant", "entropy"):
         Q = (torch.randn(heads, N, d, generator=g, device=dev) * 2).to(torch.bfloat16)
         K = torch.randn(heads, N, d, generator=g, device=dev).to(torch.bfloat16)
         V = torch.randn(heads, N, d, generator=g, device=dev).to(torch.bfloat16)
@@ -880,10 +881,24 @@ def kernel_case(args):
         elif args.case == "entropy":
             fn = lambda: tra.tra_attn_entropy(Q, K, H)  # noqa: E731
             flops = 2.0 * d * N * N * heads     # QK^T only
+        elif args.case in ("sparse_fp8", "quant"):
+            Q8 = torch.empty(heads, N, d, dtype=torch.uint8, device=dev)
+            K8 = torch.empty_like(Q8)
+            qs = torch.empty(heads, N // 128, dtype=torch.float32, device=dev)
+            ks = torch.empty_like(qs)
+            tra.tra_quantize_e4m3(Q, Q8, qs)
+            tra.tra_quantize_e4m3(K, K8, ks)
+            if args.case == "quant":
+                fn = lambda: tra.tra_quantize_e4m3(Q, Q8, qs)  # noqa: E731
+                unit = ("GB/s", heads * N * d * 3 / 1e9)    # 2 bytes read + 1 written per element
+            else:
+                fn = lambda: tra.tra_block_sparse_attn_fp8(Q8, qs, K8, ks, V, O_, rpd, cid)  # noqa: E731
+                flops = 4.0 * d * kept
         else:
             fn = lambda: tra.tra_block_sparse_attn(Q, K, V, O_, rpd, cid, 128, 128)  # noqa: E731
             flops = 4.0 * d * kept
-        unit = ("TFLOP/s", flops / 1e12)
+        if args.case != "quant":
+            unit = ("TFLOP/s", flops / 1e12)
     elif args.case == "mask":
         wl = WL
         grid = (wl.F, wl.H, wl.W)
@@ -922,7 +937,8 @@ def kernel_case(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["dense", "sparse", "entropy", "mask", "permute"], default=None,
+    ap.add_argument("--case", choices=["dense", "sparse", "sparse_fp8", "quant", "entropy", "mask",
+                                       "permute"], default=None,
                     help="run one kernel on a small case (for profiler captures)")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--workload", default="wan14b", choices=sorted(WORKLOADS) + ["sweep", "variants", "reuse"],

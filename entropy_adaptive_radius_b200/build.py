@@ -14,7 +14,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libtra.so")
-SOURCES = ["api.cu", "permute.cu", "radius.cu", "mask.cu", "attention.cu", "mask_noalloc.cu"]
+SOURCES = ["api.cu", "permute.cu", "radius.cu", "mask.cu", "attention.cu", "mask_noalloc.cu",
+           "quant.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -202,6 +202,40 @@ tra_status tra_block_sparse_attn(const void* Q, const void* K, const void* V, vo
   return status_of(launch_attention(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+tra_status tra_quantize_e4m3(const void* X, void* Xq, float* scales, int heads, int N, int d,
+                             int block, tra_stream_t stream) {
+  if (heads < 0 || N < 0) return TRA_ERR_INVALID_ARGUMENT;
+  if ((d != 64 && d != 128) || (block != 64 && block != 128)) return TRA_ERR_UNSUPPORTED;
+  if (heads == 0 || N == 0) return TRA_OK;
+  if (heads > 65535 || N > (1 << 24)) return TRA_ERR_UNSUPPORTED;
+  if (!X || !Xq || !scales || !aligned16(X) || !aligned16(Xq)) return TRA_ERR_INVALID_ARGUMENT;
+  const tra_status dv = check_device();
+  if (dv != TRA_OK) return dv;
+  return status_of(launch_quantize_e4m3(X, Xq, scales, heads, N, d, block,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tra_status tra_block_sparse_attn_fp8(const void* Q8, const float* q_scales, const void* K8,
+                                     const float* k_scales, const void* V, void* O, float* lse,
+                                     const int* row_ptr, const int* col_idx, int heads, int N,
+                                     int d, int block_q, int block_k, float scale,
+                                     tra_stream_t stream) {
+  tra_status s = check_attn_common(Q8, K8, V, O, heads, N, d, scale);
+  if (s != TRA_OK) return s;
+  if (d != 128 || block_q != 128 || block_k != 128) return TRA_ERR_UNSUPPORTED;
+  if (heads == 0 || N == 0) return TRA_OK;
+  if (!row_ptr || !col_idx || !q_scales || !k_scales) return TRA_ERR_INVALID_ARGUMENT;
+  s = check_device();
+  if (s != TRA_OK) return s;
+  AttnArgs a{};
+  a.Q = Q8; a.K = K8; a.V = V; a.O = O; a.H = nullptr; a.lse = lse;
+  a.row_ptr = row_ptr; a.col_idx = col_idx;
+  a.heads = heads; a.N = N; a.d = d; a.scale = scale; a.dense = false;
+  a.block_q = 128; a.block_k = 128;
+  a.fp8 = true; a.q_scales = q_scales; a.k_scales = k_scales;
+  return status_of(launch_attention(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 tra_status tra_budget_radius_ex(const float* H, float* r, float* phi_out, int heads,
                                 tra_grid grid, tra_tile tile, float tau, float gamma,
                                 tra_budget budget, tra_metric metric, tra_stream_t stream) {

@@ -80,6 +80,8 @@ struct Params {
   float scale_log2;
   const int* row_ptr;
   const int* col_idx;
+  const float* q_scales;  // FP8 scores: per (head, query block) scale of Q
+  const float* k_scales;  // FP8 scores: per (head, key block) scale of K
   __nv_bfloat16* O;
   float* H;
   float* lse;
@@ -629,17 +631,22 @@ static_assert(256 * kDualRegsSoftmax + 128 * kDualRegsOther == kDualThreads * kD
 static_assert(2 * kDualRegsSoftmax * 32 + kDualRegsOther * 32 <= 16384,
               "per-scheduler register file: two softmax warps and one other warp");
 
-template <int D>
+template <int D, bool FP8 = false>
 struct DualCfg {
   static constexpr int BK = 128;  // keys per super-block
   static constexpr int NS = 2;
-  static constexpr int KCH = D / 64;
-  static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BK * D * 2;
+  static constexpr int QE = FP8 ? 1 : 2;       // bytes per Q / K element
+  static constexpr int QKCH = D * QE / 128;    // 128-byte chunks of a Q / K row
+  static constexpr int QKX = 128 / QE;         // elements per chunk (TMA box width)
+  static constexpr int KSTEPS = D * QE / 32;   // MMA K-steps of QK^T (32 bytes each)
+  static constexpr int KCH = D / 64;           // 128-byte chunks of a V row (bf16)
+  static constexpr int Q_BYTES = BM * D * QE;
+  static constexpr int K_BYTES = BK * D * QE;  // one K stage
+  static constexpr int KV_BYTES = BK * D * 2;  // one V stage
   static constexpr int P_BYTES = 2 * BM * 128;  // one P_w buffer (128 rows x 128 keys bf16)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * K_BYTES;
   static constexpr int OFF_P = OFF_V + NS * KV_BYTES;  // P_0, P_1
   static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
   static constexpr int NUM_BARS = 1 + 4 * NS + 8 + 2;
@@ -650,6 +657,8 @@ struct DualCfg {
   static_assert(2 * BK + 2 * D <= TMEM_COLS, "tensor memory");
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(NUM_BARS * 8 <= 256, "barrier area");
+  static_assert(!FP8 || D == 128, "FP8 scores: one 128-byte E4M3 row per query / key");
+  static_assert(Q_BYTES % 1024 == 0 && K_BYTES % 1024 == 0, "swizzle atoms need 1 KiB alignment");
 };
 
 __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
@@ -687,12 +696,13 @@ struct ListWalker {
   }
 };
 
-template <int D, int BKS, bool DENSE>
+template <int D, int BKS, bool DENSE, bool FP8 = false>
 __global__ void __launch_bounds__(kDualThreads, 1)
     attn_dual_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Params p) {
-  using C = DualCfg<D>;
+  using C = DualCfg<D, FP8>;
+  static_assert(!FP8 || (BKS == 128 && !DENSE), "FP8 scores: block-sparse, 128-key blocks");
   constexpr int NS = C::NS;
   constexpr int BK = C::BK;
   constexpr int E = BK / BKS;  // list entries per super-block (1 or 2)
@@ -804,23 +814,24 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
 #pragma unroll
-      for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * (BM * 128), &tmQ, c * 64, qt * BM, h, bar_q);
+      for (int c = 0; c < C::QKCH; ++c)
+        tma_load_3d(sQ + c * (BM * 128), &tmQ, c * C::QKX, qt * BM, h, bar_q);
       int issued = 0;
       ListWalker wk = make_walker();
       int dn = 0;
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NS;
         if (!mbar_wait(k_empty(s), ((j / NS) & 1) ^ 1u, abort, p.err, kErrWaitKEmpty)) break;
-        mbar_arrive_expect_tx(k_full(s), C::KV_BYTES);
+        mbar_arrive_expect_tx(k_full(s), C::K_BYTES);
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           uint32_t mem;
           const int kb = next_entry(wk, dn, mem);
           const int row0 = kb >= 0 ? kb * BKS : p.N;  // past N: zeros
 #pragma unroll
-          for (int c = 0; c < C::KCH; ++c)
-            tma_load_3d(sK + s * C::KV_BYTES + c * (BK * 128) + e * BKS * 128, &tmK, c * 64, row0,
-                        h, k_full(s));
+          for (int c = 0; c < C::QKCH; ++c)
+            tma_load_3d(sK + s * C::K_BYTES + c * (BK * 128) + e * BKS * 128, &tmK, c * C::QKX,
+                        row0, h, k_full(s));
         }
         issued = j + 1;
       }
@@ -861,7 +872,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     // ===================================================== QK issuer (block order)
     // QK_j needs K_j and the release of S_{j mod 2} by block j - 2's softmax.
     if (lane == 0) {
-      constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BK, 0, 0);
+      constexpr uint32_t kIdescQK = FP8 ? idesc_e4m3_f32(BM, BK) : idesc_bf16_f32(BM, BK, 0, 0);
       bool ok = mbar_wait(bar_q, 0, abort, p.err, kErrWaitQ);
       for (int j = 0; ok && j < nblk; ++j) {
         const int s = j % NS, w = j & 1, i = j >> 1;
@@ -870,12 +881,17 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t tS = tmem + w * BK;
+        // K-steps of 32 bytes (16 bf16 or 32 E4M3 elements) along the rows
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < C::KSTEPS; ++k) {
           const uint64_t a = smem_desc_sw128(sQ + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024);
           const uint64_t bd =
-              smem_desc_sw128(sK + s * C::KV_BYTES + (k >> 2) * (BK * 128) + (k & 3) * 32, 16, 1024);
-          mma_bf16_ss(tS, a, bd, kIdescQK, k > 0 ? 1u : 0u);
+              smem_desc_sw128(sK + s * C::K_BYTES + (k >> 2) * (BK * 128) + (k & 3) * 32, 16, 1024);
+          if constexpr (FP8) {
+            mma_f8_ss(tS, a, bd, kIdescQK, k > 0 ? 1u : 0u);
+          } else {
+            mma_bf16_ss(tS, a, bd, kIdescQK, k > 0 ? 1u : 0u);
+          }
         }
         mma_commit(k_empty(s));
         mma_commit(s_full(w));
@@ -946,13 +962,21 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     // entry, so entry j is simply the j-th list element (one load, no walk)
     const bool direct = (E == 1) && (DENSE || p.G == 1);
     const int* my_list = p.col_idx + misc[3];
+    // FP8 scores carry the query block's and the key block's scale
+    float q_sl2 = p.scale_log2;
+    if constexpr (FP8) q_sl2 *= __ldg(p.q_scales + static_cast<size_t>(h) * p.nqb + qt);
     for (int i = 0; i < nmine; ++i) {
       const int j = 2 * i + w;
       // valid keys of each entry of super-block j for this row
       int nv[E];
+      float sl2 = q_sl2;
       if (direct) {
         const int kb = DENSE ? j : __ldg(my_list + j);
-        nv[0] = (kb >= 0 && kb < p.nkb) ? min(BKS, p.N - kb * BKS) : 0;
+        const bool kb_ok = kb >= 0 && kb < p.nkb;
+        nv[0] = kb_ok ? min(BKS, p.N - kb * BKS) : 0;
+        if constexpr (FP8) {
+          if (kb_ok) sl2 *= __ldg(p.k_scales + static_cast<size_t>(h) * p.nkb + kb);
+        }
       } else {
         // walk the merged list, skipping the other warpgroup's super-blocks
         for (; sb_done < j; ++sb_done) {
@@ -1060,12 +1084,12 @@ __global__ void __launch_bounds__(kDualThreads, 1)
           for (int q = 0; q < 5; ++q) mx[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
           const float m6 = fmax3(mx[0], mx[1], mx[2]);
           const float m7 = fmax3(mx[3], mx[4], mx[15]);
-          if (any_valid) update_max(fmaxf(m6, m7) * p.scale_log2);
+          if (any_valid) update_max(fmaxf(m6, m7) * sl2);
         }
         // x = s * scale * log2(e) - m_ref, p = 2^x, Z += p, A += p * x, two
         // lanes per instruction (m_ref is -inf only for a row with no valid
         // key yet, whose p are then all 0)
-        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 sc2 = make_float2(sl2, sl2);
         const float mc = (m_ref == -INFINITY) ? 0.f : m_ref;
         const float2 nm2 = make_float2(-mc, -mc);
         float2 z2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -1438,28 +1462,31 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [heads, N, d] bf16 as a 3D tensor (d, N, heads); boxes of 64 x rows x 1,
-// 128-byte swizzle; rows past N read as zeros.
-bool make_map(CUtensorMap* map, const void* base, int d, int N, int heads, int rows) {
+// [heads, N, d] as a 3D tensor (d, N, heads) of bf16 (esize 2) or E4M3 bytes
+// (esize 1); boxes of (128 / esize) x rows x 1, i.e. 128-byte rows, 128-byte
+// swizzle; rows past N read as zeros.
+bool make_map(CUtensorMap* map, const void* base, int d, int N, int heads, int rows,
+              int esize = 2) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                               static_cast<cuuint64_t>(heads)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                                 static_cast<cuuint64_t>(N) * d * 2};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize,
+                                 static_cast<cuuint64_t>(N) * d * esize};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esize), static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+  const CUresult r = fn(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                        3, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BKS, bool DENSE>
+template <int D, int BKS, bool DENSE, bool FP8 = false>
 cudaError_t launch_dual(const AttnArgs& a, const Params& prm, cudaStream_t stream) {
-  using C = DualCfg<D>;
-  auto kern = attn_dual_kernel<D, BKS, DENSE>;
+  using C = DualCfg<D, FP8>;
+  auto kern = attn_dual_kernel<D, BKS, DENSE, FP8>;
   // The kernel's register split assumes exactly kDualLaunchRegs per thread at
   // launch; with any other allocation setmaxnreg.inc could wait forever.
   static const int launch_regs = [kern] {
@@ -1468,7 +1495,8 @@ cudaError_t launch_dual(const AttnArgs& a, const Params& prm, cudaStream_t strea
   }();
   if (launch_regs != kDualLaunchRegs) return cudaErrorInvalidDeviceFunction;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, a.Q, D, a.N, a.heads, BM) || !make_map(&mk, a.K, D, a.N, a.heads, BKS) ||
+  if (!make_map(&mq, a.Q, D, a.N, a.heads, BM, C::QE) ||
+      !make_map(&mk, a.K, D, a.N, a.heads, BKS, C::QE) ||
       !make_map(&mv, a.V, D, a.N, a.heads, BKS))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -1521,6 +1549,8 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
   prm.scale_log2 = a.scale * kLog2e;
   prm.row_ptr = a.row_ptr;
   prm.col_idx = a.col_idx;
+  prm.q_scales = a.q_scales;
+  prm.k_scales = a.k_scales;
   prm.O = static_cast<__nv_bfloat16*>(a.O);
   prm.H = a.H;
   prm.lse = a.lse;
@@ -1530,6 +1560,8 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
   // which merges the lists of up to eight query blocks per CTA.
   if (a.entropy_only) return a.d == 128 ? launch_entropy<128>(a, prm, stream)
                                           : launch_entropy<64>(a, prm, stream);
+  // E4M3 Q and K: 128-row query blocks, 128-key blocks, d = 128 (checked by the API)
+  if (a.fp8) return launch_dual<128, 128, false, true>(a, prm, stream);
   if (a.dense) {
     if (a.d == 128) return launch_dual<128, 128, true>(a, prm, stream);
     return launch_dual<64, 128, true>(a, prm, stream);

@@ -64,7 +64,13 @@ struct AttnArgs {
   float scale;
   bool dense;
   bool entropy_only;  // H (and LSE) over all keys, no output (V and O unused)
+  bool fp8;           // Q and K are E4M3 codes with per-block scales
+  const float* q_scales;  // [heads, ceil(N / 128)] (fp8 only)
+  const float* k_scales;  // [heads, ceil(N / 128)] (fp8 only)
 };
+// quant.cu: per (head, block of `block` rows) E4M3 quantization of bf16 X
+cudaError_t launch_quantize_e4m3(const void* X, void* Xq, float* scales, int heads, int N, int d,
+                                 int block, cudaStream_t stream);
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace tra

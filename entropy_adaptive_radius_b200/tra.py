@@ -66,6 +66,9 @@ _PROTOS = {
                                               _vp, _vp, _c_ll, _vp, _vp]),
     "tra_block_sparse_attn": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                                        _c_int, _c_int, _c_float, _vp]),
+    "tra_quantize_e4m3": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp]),
+    "tra_block_sparse_attn_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int,
+                                           _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
     "tra_get_device_error": (_c_int, [ctypes.POINTER(_c_int), _vp]),
 }
 
@@ -256,6 +259,30 @@ def tra_block_sparse_attn(Q, K, V, O, row_ptr, col_idx, block_q, block_k, lse=No
     _check("tra_block_sparse_attn", lib().tra_block_sparse_attn(
         _p(Q), _p(K), _p(V), _p(O), _p(lse), _p(row_ptr), _p(col_idx), heads, N, d, block_q,
         block_k, scale, _stream(stream)))
+    return O
+
+
+def tra_quantize_e4m3(X, Xq, scales, block=128, stream=None):
+    """Per-block E4M3 codes Xq (uint8 [heads, N, d]) and fp32 scales
+    [heads, ceil(N / block)] of a bf16 X [heads, N, d]."""
+    _contig(X, Xq, scales)
+    heads, N, d = X.shape
+    if Xq.dtype != torch.uint8:
+        raise TypeError("Xq holds E4M3 codes as uint8")
+    _check("tra_quantize_e4m3", lib().tra_quantize_e4m3(
+        _p(X), _p(Xq), _p(scales), heads, N, d, block, _stream(stream)))
+    return Xq, scales
+
+
+def tra_block_sparse_attn_fp8(Q8, q_scales, K8, k_scales, V, O, row_ptr, col_idx, block_q=128,
+                              block_k=128, lse=None, scale=None, stream=None):
+    """Block-sparse attention with E4M3 Q and K (from tra_quantize_e4m3, block 128)."""
+    _contig(Q8, q_scales, K8, k_scales, V, O, row_ptr, col_idx, lse)
+    heads, N, d = V.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    _check("tra_block_sparse_attn_fp8", lib().tra_block_sparse_attn_fp8(
+        _p(Q8), _p(q_scales), _p(K8), _p(k_scales), _p(V), _p(O), _p(lse), _p(row_ptr),
+        _p(col_idx), heads, N, d, block_q, block_k, scale, _stream(stream)))
     return O
 
 

@@ -312,6 +312,39 @@ tra_status tra_block_sparse_attn(const void* Q, const void* K, const void* V, vo
                                  tra_stream_t stream);
 
 /*
+ * ---- FP8 scores -----------------------------------------------------------
+ * The block-sparse call with QK^T on the tensor cores' 8-bit (E4M3) kind:
+ * same mask, same exact softmax over the kept blocks, PV still in bf16.  The
+ * pages fix no precision; the quantization below is this library's reading.
+ *
+ * Per-block E4M3 quantization of a bf16 tensor.  For every head and every
+ * block of `block` consecutive rows: amax = max |x| over the block,
+ * scale = fl32(amax / 448) (1 for an all-zero block), and
+ * Xq = E4M3(fl32(x / scale)) (OCP FP8 E4M3, ties to even, saturating).
+ *   X       [heads, N, d] bf16, 16-byte aligned; read only.
+ *   Xq      [heads, N, d] bytes (E4M3 codes), 16-byte aligned; written.
+ *   scales  [heads, ceil(N / block)] fp32; written.
+ *   d in {64, 128}; block in {64, 128}.
+ */
+tra_status tra_quantize_e4m3(const void* X, void* Xq, float* scales, int heads, int N, int d,
+                             int block, tra_stream_t stream);
+
+/*
+ * tra_block_sparse_attn with E4M3 queries and keys: the score of query i and
+ * key j is scale * q_scales[i / 128] * k_scales[j / 128] * (q8_i . k8_j),
+ * accumulated in fp32 on the tensor cores; the rest is tra_block_sparse_attn.
+ *   Q8, K8    [heads, N, 128] E4M3 codes from tra_quantize_e4m3 with block 128.
+ *   q_scales, k_scales  [heads, ceil(N / 128)] fp32 from the same call.
+ *   V, O, lse, row_ptr, col_idx, scale: as for tra_block_sparse_attn.
+ *   d = 128 and block_q = block_k = 128 only (TRA_ERR_UNSUPPORTED otherwise).
+ */
+tra_status tra_block_sparse_attn_fp8(const void* Q8, const float* q_scales, const void* K8,
+                                     const float* k_scales, const void* V, void* O, float* lse,
+                                     const int* row_ptr, const int* col_idx, int heads, int N,
+                                     int d, int block_q, int block_k, float scale,
+                                     tra_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word of the
  * current device.  *code = 0 when no kernel recorded an error; otherwise the
  * code of the first wait that ran out of time.  Returns TRA_ERR_TIMEOUT when

@@ -155,3 +155,19 @@ def test_variant_validation(L):
     assert m(P, P, 40, G, T, 128, 128, 1, 7, P, P, 100, P, P, ws, S0) == INVALID
     assert m(P, P, 40, G, T, 128, 48, 1, 1, P, P, 100, P, P, ws, S0) == UNSUPPORTED
     assert m(P, P, 40, G, T, 128, 128, 1, 1, P, P, 100, P, P, ws - 1, S0) == WORKSPACE
+
+
+def test_fp8_validation(L):
+    q = L.tra_quantize_e4m3
+    assert q(P, P2, P, 2, 1000, 96, 128, S0) == UNSUPPORTED
+    assert q(P, P2, P, 2, 1000, 128, 32, S0) == UNSUPPORTED
+    assert q(None, P2, P, 2, 1000, 128, 128, S0) == INVALID
+    assert q(P, MIS, P, 2, 1000, 128, 128, S0) == INVALID
+    assert q(P, P2, None, 2, 1000, 128, 128, S0) == INVALID
+    assert q(None, None, None, 0, 1000, 128, 128, S0) == OK
+    a = L.tra_block_sparse_attn_fp8
+    assert a(P, P, P, P, P, P, None, P, P, 2, 1000, 64, 128, 128, 0.1, S0) == UNSUPPORTED
+    assert a(P, P, P, P, P, P, None, P, P, 2, 1000, 128, 64, 64, 0.1, S0) == UNSUPPORTED
+    assert a(P, None, P, P, P, P, None, P, P, 2, 1000, 128, 128, 128, 0.1, S0) == INVALID
+    assert a(P, P, P, P, P, P, None, None, P, 2, 1000, 128, 128, 128, 0.1, S0) == INVALID
+    assert a(P, P, P, P, P, P, None, P, P, 2, 1000, 128, 128, 128, 0.0, S0) == INVALID
