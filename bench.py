@@ -526,68 +526,76 @@ def gpu_arm(args, rank, world, local):
 
 
 def e2e_run(pipe, host, dev, calls, args, device, world):
-    """End to end through the C ABI from pinned host memory: every call's
-    inputs (Q, K, V in original order) are copied host -> device and its
-    output O device -> host inside the timed region.  Copies in and copies out
-    run on two streams of their own (so both copy engines work at once) into
-    double buffers: the next call's inputs and the previous call's output move
-    while the current call computes."""
+    """End to end through the C ABI from pinned host memory.  Every step's
+    inputs (its distinct tensors: Q, K, V of the warm-up call and Q_c, K_c of
+    each sparse call, V being shared, all in the original token order) are
+    copied host -> device, and every call's output O device -> host, inside
+    the timed region.  Inputs are double-buffered per step on a copy-in
+    stream, so the next step's inputs move while this step computes; outputs
+    go back on a copy-out stream (the two directions run at once)."""
     comp = torch.cuda.current_stream(device)
     cin, cout = torch.cuda.Stream(device), torch.cuda.Stream(device)
-    slots = [[torch.empty_like(dev[0]) for _ in range(3)] for _ in range(2)]
-    outs = [torch.empty_like(pipe.O) for _ in range(2)]
-    out_host = [torch.empty(pipe.O.shape, dtype=pipe.O.dtype).pin_memory() for _ in range(2)]
-    ready = [torch.cuda.Event() for _ in range(2)]
-    done = [torch.cuda.Event() for _ in range(2)]
-    copied_out = [torch.cuda.Event() for _ in range(2)]
-    # one step = warm-up call on (Q, K, V), then `calls` sparse calls on (Q_c, K_c, V)
-    step_inputs = [(host[0], host[1], host[2])] + [(host[3 + 2 * c], host[4 + 2 * c], host[2])
-                                                  for c in range(calls)]
-    nbytes_in = sum(x.numel() * x.element_size() for tr in step_inputs for x in tr)
-    nbytes_out = len(step_inputs) * out_host[0].numel() * out_host[0].element_size()
-    started = [False, False]
+    n_in = len(host)                        # 3 + 2 * calls distinct inputs
+    sets = [[torch.empty_like(dev[i]) for i in range(n_in)] for _ in range(2)]
+    outs = [[torch.empty_like(pipe.O) for _ in range(calls + 1)] for _ in range(2)]
+    out_host = [torch.empty(pipe.O.shape, dtype=pipe.O.dtype).pin_memory() for _ in range(calls + 1)]
+    ready = [[torch.cuda.Event() for _ in range(calls + 1)] for _ in range(2)]
+    copied = [[torch.cuda.Event() for _ in range(calls + 1)] for _ in range(2)]
+    step_done = [torch.cuda.Event(), torch.cuda.Event()]
+    used = [False, False]
+    # inputs of call c: (Q, K, V) for the warm-up, (Q_c, K_c, V) after it
+    call_in = [(0, 1, 2)] + [(3 + 2 * c, 4 + 2 * c, 2) for c in range(calls)]
+    nbytes_in = sum(x.numel() * x.element_size() for x in host)
+    nbytes_out = (calls + 1) * out_host[0].numel() * out_host[0].element_size()
 
-    def h2d(k, slot):
-        srcs = step_inputs[k % len(step_inputs)]
+    def copy_in(st):
         with torch.cuda.stream(cin):
-            if started[slot]:
-                cin.wait_event(done[slot])       # the call that used this slot is finished
-            for d_, s_ in zip(slots[slot], srcs):
-                d_.copy_(s_, non_blocking=True)
-            ready[slot].record(cin)
+            if used[st]:
+                cin.wait_event(step_done[st])   # the step that last used this set is done
+            done = set()
+            for c, idx in enumerate(call_in):
+                for i in idx:
+                    if i not in done:
+                        sets[st][i].copy_(host[i], non_blocking=True)
+                        done.add(i)
+                ready[st][c].record(cin)
 
-    def run(total):
-        h2d(0, 0)
-        for k in range(total):
-            slot = k % 2
-            if k + 1 < total:
-                h2d(k + 1, (k + 1) % 2)
-            comp.wait_event(ready[slot])
-            if started[slot]:
-                comp.wait_event(copied_out[slot])  # output buffer of this slot was read back
-            q, kk, v = slots[slot]
-            if k % len(step_inputs) == 0:
-                pipe.warmup_call(q, kk, v, None, out=outs[slot])
+    def compute(st):
+        for c, (iq, ik, iv) in enumerate(call_in):
+            comp.wait_event(ready[st][c])
+            if used[st]:
+                comp.wait_event(copied[st][c])  # this output buffer has been read back
+            q, k, v = sets[st][iq], sets[st][ik], sets[st][iv]
+            if c == 0:
+                pipe.warmup_call(q, k, v, None, out=outs[st][c])
             else:
-                pipe.sparse_call(q, kk, v, None, out=outs[slot])
-            done[slot].record(comp)
-            started[slot] = True
+                pipe.sparse_call(q, k, v, None, out=outs[st][c])
+            ev = torch.cuda.Event()
+            ev.record(comp)
             with torch.cuda.stream(cout):
-                cout.wait_event(done[slot])
-                out_host[slot].copy_(outs[slot], non_blocking=True)
-                copied_out[slot].record(cout)
+                cout.wait_event(ev)
+                out_host[c].copy_(outs[st][c], non_blocking=True)
+                copied[st][c].record(cout)
+        step_done[st].record(comp)
+        used[st] = True
+
+    def run(n):
+        copy_in(0)
+        for k in range(n):
+            if k + 1 < n:
+                copy_in((k + 1) % 2)
+            compute(k % 2)
         comp.wait_stream(cout)
 
-    run(len(step_inputs))   # warm-up
+    run(2)   # warm-up
     torch.cuda.synchronize()
-    started[0] = started[1] = False
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    steps = max(1, min(args.steps, 3))
+    steps = max(2, min(args.steps, 4))
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record(comp)
-    run(steps * len(step_inputs))
+    run(steps)
     e.record(comp)
     torch.cuda.synchronize()
     ms = s.elapsed_time(e)
