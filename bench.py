@@ -343,8 +343,10 @@ def gpu_arm(args, rank, world, local):
     torch.cuda.set_device(device)
     log = (lambda m: print(f"[bench] {m}", file=sys.stderr, flush=True)) if rank == 0 else (lambda m: None)
     if world > 1:
+        # short enough that ranks waiting on a lost rank fail soon; the longest
+        # gap between two collectives here is well under a minute
         dist.init_process_group("nccl", device_id=device,
-                                timeout=__import__("datetime").timedelta(seconds=600))
+                                timeout=__import__("datetime").timedelta(seconds=180))
     wl = WORKLOADS[args.workload]
     calls = wl.sparse_calls
     t0 = time.time()
