@@ -696,7 +696,7 @@ struct ListWalker {
   }
 };
 
-template <int D, int BKS, bool DENSE, bool FP8 = false>
+template <int D, int BKS, bool DENSE, bool FP8 = false, bool SINGLE = true>
 __global__ void __launch_bounds__(kDualThreads, 1)
     attn_dual_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
@@ -956,11 +956,11 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     // the CTA (rows 64g .. 64g+63 when two 64-row query blocks share it)
     ListWalker wk = make_walker();
     int dn = 0, sb_done = 0;
-    const uint32_t my_bit = (p.G == 2) ? (1u << (row >> 6)) : 1u;
+    const uint32_t my_bit = SINGLE ? 1u : (1u << (row >> 6));
     // One query block per CTA and one list entry per super-block (128-row
     // query blocks, 128-key blocks, and the dense pass): every row keeps every
     // entry, so entry j is simply the j-th list element (one load, no walk)
-    const bool direct = (E == 1) && (DENSE || p.G == 1);
+    constexpr bool kDirect = (E == 1) && (DENSE || SINGLE);
     const int* my_list = p.col_idx + misc[3];
     // FP8 scores carry the query block's and the key block's scale
     float q_sl2 = p.scale_log2;
@@ -970,7 +970,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       // valid keys of each entry of super-block j for this row
       int nv[E];
       float sl2 = q_sl2;
-      if (direct) {
+      if constexpr (kDirect) {
         const int kb = DENSE ? j : __ldg(my_list + j);
         const bool kb_ok = kb >= 0 && kb < p.nkb;
         nv[0] = kb_ok ? min(BKS, p.N - kb * BKS) : 0;
@@ -1029,8 +1029,11 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       };
       // Three cases, warp-uniform: every key of the block valid for the whole
       // warp (fast path), none valid (P = 0), or a partly valid tail block.
-      const int mode = __all_sync(0xffffffffu, all_valid) ? 0
-                       : (__all_sync(0xffffffffu, !any_valid) ? 1 : 2);
+      // (with one query block per tile every row has the same valid keys)
+      const int mode = kDirect ? (all_valid ? 0 : (any_valid ? 2 : 1))
+                       : (__all_sync(0xffffffffu, all_valid)
+                              ? 0
+                              : (__all_sync(0xffffffffu, !any_valid) ? 1 : 2));
       auto wait_prev_pv = [&]() -> bool {
         // P_w and O_w are free once this warpgroup's previous PV has completed
         if (i > 0) {
@@ -1483,10 +1486,10 @@ bool make_map(CUtensorMap* map, const void* base, int d, int N, int heads, int r
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BKS, bool DENSE, bool FP8 = false>
+template <int D, int BKS, bool DENSE, bool FP8 = false, bool SINGLE = true>
 cudaError_t launch_dual(const AttnArgs& a, const Params& prm, cudaStream_t stream) {
   using C = DualCfg<D, FP8>;
-  auto kern = attn_dual_kernel<D, BKS, DENSE, FP8>;
+  auto kern = attn_dual_kernel<D, BKS, DENSE, FP8, SINGLE>;
   // The kernel's register split assumes exactly kDualLaunchRegs per thread at
   // launch; with any other allocation setmaxnreg.inc could wait forever.
   static const int launch_regs = [kern] {
@@ -1567,11 +1570,19 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
     return launch_dual<64, 128, true>(a, prm, stream);
   }
   if ((bq == 128 || bq == 64) && (bk == 128 || bk == 64)) {
+    // SINGLE: one query block per 128-row tile
+    if (bq == 128) {
+      if (a.d == 128)
+        return bk == 128 ? launch_dual<128, 128, false, false, true>(a, prm, stream)
+                         : launch_dual<128, 64, false, false, true>(a, prm, stream);
+      return bk == 128 ? launch_dual<64, 128, false, false, true>(a, prm, stream)
+                       : launch_dual<64, 64, false, false, true>(a, prm, stream);
+    }
     if (a.d == 128)
-      return bk == 128 ? launch_dual<128, 128, false>(a, prm, stream)
-                       : launch_dual<128, 64, false>(a, prm, stream);
-    return bk == 128 ? launch_dual<64, 128, false>(a, prm, stream)
-                     : launch_dual<64, 64, false>(a, prm, stream);
+      return bk == 128 ? launch_dual<128, 128, false, false, false>(a, prm, stream)
+                       : launch_dual<128, 64, false, false, false>(a, prm, stream);
+    return bk == 128 ? launch_dual<64, 128, false, false, false>(a, prm, stream)
+                     : launch_dual<64, 64, false, false, false>(a, prm, stream);
   }
   if (a.d == 128) {
     if (bk == 128) return launch_cfg<128, 128, false>(a, prm, stream);
