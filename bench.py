@@ -121,6 +121,19 @@ def max_over_ranks(value_ms, device=None):
     return float(t.item())
 
 
+def workload_config(wl, world, tau=None, kept=None):
+    """The `config` object of the JSON line, the same for both arms: the
+    workload and its shape; tau and the kept fraction as measured (the GPU
+    arm calibrates tau to the workload's target) or the target itself."""
+    return {"workload": wl.name, "grid": [wl.F, wl.H, wl.W], "N": wl.N, "heads": wl.heads,
+            "head_dim": wl.d, "block": [wl.block_q, wl.block_k], "tile": list(wl.tile),
+            "gamma": wl.gamma, "vote": wl.vote,
+            "tau": None if tau is None else round(tau, 6),
+            "kept_fraction": None if kept is None else round(kept, 4),
+            "sparse_calls_per_warmup": wl.sparse_calls, "l2": l2_note(wl),
+            "parallelism": f"independent x{world}"}
+
+
 def kept_pair_tokens(row_ptr, col_idx, heads, N, bq, bk):
     """sum over kept (qb, kb) of |qb| * |kb| (tail blocks shorter), all heads."""
     nqb, nkb = -(-N // bq), -(-N // bk)
@@ -488,11 +501,7 @@ def gpu_arm(args, rank, world, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Fourier-feature Q/K of grid position + noise, v ~ N(0,1))",
-        "config": {"workload": wl.name, "grid": [wl.F, wl.H, wl.W], "N": wl.N, "heads": wl.heads,
-                   "head_dim": wl.d, "block": [wl.block_q, wl.block_k], "tile": list(wl.tile),
-                   "gamma": wl.gamma, "vote": wl.vote, "tau": round(pipe.tau, 6),
-                   "kept_fraction": round(kept, 4), "sparse_calls_per_warmup": calls,
-                   "l2": l2_note(wl), "parallelism": f"independent x{world}"},
+        "config": workload_config(wl, world, tau=pipe.tau, kept=kept),
         "sparse_ms_per_call": round(s_ms, 3), "sparse_tflops_kept": round(sparse_tf, 2),
         "dense_ms_per_call": round(d_ms, 3), "dense_tflops": round(dense_tf, 2),
         "mask_ms": round(statistics.mean(mask_ms), 3), "radius_ms": round(statistics.mean(radius_ms), 4),
@@ -852,7 +861,7 @@ def reference_arm(args, rank, world):
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(t * 1e3, 1), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": wl.name, "kept_fraction": kept},
+           "config": workload_config(wl, world, kept=kept),
            "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": host_threads(),
                             "kind": "oracle", "sample": sample},
            "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
