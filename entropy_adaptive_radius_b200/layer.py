@@ -17,6 +17,13 @@ kind of step it is follows the `ReusePolicy`:
     an entropy-only pass (no PV product); `refresh = "dense"` makes the step a
     dense one.
 
+The mask may also come from the variants the summary's §4 ablations and
+Radial Attention describe: `budget="shared"` gives every query of a head the
+head's mean budget, `metric="line"` measures distance along the in-frame
+raster order, and `radial_r0=r0` replaces the entropy by Radial Attention's
+static window (base radius r0, window halving per doubling of the temporal
+distance); the sparse steps are unchanged.
+
 With `layout="tile_major"` the layer takes and returns tensors that are
 already in tile-major order and runs no permutation: a model that keeps the
 tokens of a whole transformer block in tile-major order permutes once on the
@@ -63,10 +70,17 @@ class TraLayer:
 
     def __init__(self, grid: Sequence[int], heads: int, d: int, *, tau: float, gamma: float,
                  tile=(1, 4, 4), block_q: int = 128, block_k: int = 128, vote: int = 1,
-                 policy: ReusePolicy = ReusePolicy(), layout: str = "original", device="cuda"):
+                 policy: ReusePolicy = ReusePolicy(), layout: str = "original",
+                 budget: str = "entropy", metric: str = "disk", radial_r0: Optional[float] = None,
+                 device="cuda"):
         if layout not in ("original", "tile_major"):
             raise ValueError("layout is 'original' or 'tile_major'")
+        if budget not in tra.BUDGETS or metric not in tra.METRICS:
+            raise ValueError("budget is 'entropy' or 'shared'; metric is 'disk' or 'line'")
+        if radial_r0 is not None and not radial_r0 >= 0:
+            raise ValueError("radial_r0 >= 0")
         self.layout = layout
+        self.budget, self.metric, self.radial_r0 = budget, metric, radial_r0
         self.grid = tuple(int(v) for v in grid)
         F, H, W = self.grid
         self.N = F * H * W
@@ -98,11 +112,15 @@ class TraLayer:
         self.step_index = 0
 
     def _rebuild_mask(self):
-        tra.tra_budget_radius(self.H, self.r, self.grid, self.tau, self.gamma, self.tile,
-                              phi_out=self.phi)
-        tra.tra_build_block_mask(self.r, self.phi, self.grid, self.block_q, self.block_k,
-                                 self.vote, self.row_ptr, self.col_idx, self.nnz, self.ws,
-                                 self.tile)
+        if self.radial_r0 is not None:
+            tra.tra_radial_radius(self.r, self.grid, self.radial_r0, self.metric, self.tile,
+                                  phi_out=self.phi)
+        else:
+            tra.tra_budget_radius_ex(self.H, self.r, self.grid, self.tau, self.gamma, self.budget,
+                                     self.metric, self.tile, phi_out=self.phi)
+        tra.tra_build_block_mask_ex(self.r, self.phi, self.grid, self.block_q, self.block_k,
+                                    self.vote, self.row_ptr, self.col_idx, self.nnz, self.ws,
+                                    self.metric, self.tile)
 
     def to_tile_major(self, X: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
         """[heads, N, d] from the original token order to tile-major order (bf16)."""

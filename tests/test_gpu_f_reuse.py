@@ -136,3 +136,35 @@ def test_tile_major_resident_layer_matches_original_layout():
     assert tra.tra_get_device_error() == 0
     with pytest.raises(ValueError):
         TraLayer((F, HH, WW), HEADS, D, layout="diagonal", **kw)
+
+
+@pytest.mark.parametrize("budget,metric,r0", [("shared", "disk", None), ("entropy", "line", None),
+                                              ("entropy", "disk", 2.5), ("entropy", "line", 9.0)])
+def test_layer_mask_variants_match_the_component_calls(budget, metric, r0):
+    """The layer's variant masks are the ones the variant entry points build
+    from its own entropy (the components are pinned to the oracle in
+    test_gpu_d_variants); the sparse steps then use them."""
+    need_gpu()
+    steps = make_steps(seed=11)
+    layer = TraLayer((F, HH, WW), HEADS, D, tau=0.1, gamma=GAMMA, tile=TILE, block_q=BQ, block_k=BK,
+                     budget=budget, metric=metric, radial_r0=r0)
+    Q, K, V = (x.cuda() for x in steps[0])
+    layer(Q, K, V)
+    grid = (F, HH, WW)
+    r = torch.empty_like(layer.H)
+    phi = torch.empty(F, dtype=torch.float32, device="cuda")
+    if r0 is None:
+        tra.tra_budget_radius_ex(layer.H, r, grid, 0.1, GAMMA, budget, metric, TILE, phi_out=phi)
+    else:
+        tra.tra_radial_radius(r, grid, r0, metric, TILE, phi_out=phi)
+    nqb = -(-N // BQ)
+    rp = torch.empty(HEADS * (nqb + 1), dtype=torch.int32, device="cuda")
+    ci = torch.empty(HEADS * nqb * nqb, dtype=torch.int32, device="cuda")
+    nnz = torch.empty(1, dtype=torch.int32, device="cuda")
+    ws = tra.workspace_tensor(tra.tra_mask_workspace_size(HEADS, grid, BQ, BK, TILE))
+    tra.tra_build_block_mask_ex(r, phi, grid, BQ, BK, 1, rp, ci, nnz, ws, metric, TILE)
+    n = int(nnz.item())
+    assert n == int(layer.nnz.item()) and torch.equal(rp, layer.row_ptr)
+    assert torch.equal(ci[:n], layer.col_idx[:n])
+    O1 = layer(*(x.cuda() for x in steps[1]))            # a sparse step over that mask
+    assert tra.tra_get_device_error() == 0 and bool(torch.isfinite(O1.float()).all())
