@@ -15,7 +15,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libtra.so")
 SOURCES = ["api.cu", "permute.cu", "radius.cu", "mask.cu", "attention.cu", "mask_noalloc.cu",
-           "quant.cu"]
+           "quant.cu", "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

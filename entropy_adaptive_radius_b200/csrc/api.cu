@@ -8,9 +8,18 @@
 #include <cstdint>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "tra_internal.h"
 
 namespace tra {
+
+// One NVTX range per API call (named after the call), visible to Nsight
+// tools; with no tool attached the calls do nothing.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 // Device error word: first code recorded by a kernel whose wait ran out of time.
 __device__ int g_device_error = 0;
@@ -102,6 +111,7 @@ int tra_version(void) { return 100; }
 tra_status tra_tile_major_permute(const void* X, void* X_tm, tra_dtype in_dtype,
                                   tra_dtype out_dtype, int heads, int d, tra_grid grid,
                                   tra_tile tile, tra_stream_t stream) {
+  NvtxRange nvtx_range("tra_tile_major_permute");
   if (heads < 0 || !grid_ok(grid) || !tile_ok(tile)) return TRA_ERR_INVALID_ARGUMENT;
   if ((in_dtype != TRA_BF16 && in_dtype != TRA_F32) || (out_dtype != TRA_BF16 && out_dtype != TRA_F32))
     return TRA_ERR_INVALID_ARGUMENT;
@@ -120,6 +130,7 @@ tra_status tra_tile_major_permute(const void* X, void* X_tm, tra_dtype in_dtype,
 
 tra_status tra_inverse_permute(const void* X_tm, void* X, tra_dtype dtype, int heads, int d,
                                tra_grid grid, tra_tile tile, tra_stream_t stream) {
+  NvtxRange nvtx_range("tra_inverse_permute");
   if (heads < 0 || !grid_ok(grid) || !tile_ok(tile)) return TRA_ERR_INVALID_ARGUMENT;
   if (dtype != TRA_BF16 && dtype != TRA_F32) return TRA_ERR_INVALID_ARGUMENT;
   if (d < 8 || d > 1024 || d % 8 != 0) return TRA_ERR_UNSUPPORTED;
@@ -151,6 +162,7 @@ static tra_status check_attn_common(const void* Q, const void* K, const void* V,
 tra_status tra_dense_attn_entropy(const void* Q, const void* K, const void* V, void* O, float* H,
                                   float* lse, int heads, int N, int d, float scale,
                                   tra_stream_t stream) {
+  NvtxRange nvtx_range("tra_dense_attn_entropy");
   tra_status s = check_attn_common(Q, K, V, O, heads, N, d, scale);
   if (s != TRA_OK || heads == 0 || N == 0) return s;
   if (H == nullptr) return TRA_ERR_INVALID_ARGUMENT;
@@ -165,6 +177,7 @@ tra_status tra_dense_attn_entropy(const void* Q, const void* K, const void* V, v
 
 tra_status tra_attn_entropy(const void* Q, const void* K, float* H, float* lse, int heads, int N,
                             int d, float scale, tra_stream_t stream) {
+  NvtxRange nvtx_range("tra_attn_entropy");
   if (heads < 0 || N < 0) return TRA_ERR_INVALID_ARGUMENT;
   if (!(scale > 0.f) || !std::isfinite(scale)) return TRA_ERR_INVALID_ARGUMENT;
   if (d != 64 && d != 128) return TRA_ERR_UNSUPPORTED;
@@ -183,6 +196,7 @@ tra_status tra_attn_entropy(const void* Q, const void* K, float* H, float* lse, 
 tra_status tra_block_sparse_attn(const void* Q, const void* K, const void* V, void* O, float* lse,
                                  const int* row_ptr, const int* col_idx, int heads, int N, int d,
                                  int block_q, int block_k, float scale, tra_stream_t stream) {
+  NvtxRange nvtx_range("tra_block_sparse_attn");
   tra_status s = check_attn_common(Q, K, V, O, heads, N, d, scale);
   if (s != TRA_OK) return s;
   if (!block_ok(block_q) || !block_ok(block_k)) return TRA_ERR_UNSUPPORTED;
@@ -204,6 +218,7 @@ tra_status tra_block_sparse_attn(const void* Q, const void* K, const void* V, vo
 
 tra_status tra_quantize_e4m3(const void* X, void* Xq, float* scales, int heads, int N, int d,
                              int block, tra_stream_t stream) {
+  NvtxRange nvtx_range("tra_quantize_e4m3");
   if (heads < 0 || N < 0) return TRA_ERR_INVALID_ARGUMENT;
   if ((d != 64 && d != 128) || (block != 64 && block != 128)) return TRA_ERR_UNSUPPORTED;
   if (heads == 0 || N == 0) return TRA_OK;
@@ -220,6 +235,7 @@ tra_status tra_block_sparse_attn_fp8(const void* Q8, const float* q_scales, cons
                                      const int* row_ptr, const int* col_idx, int heads, int N,
                                      int d, int block_q, int block_k, float scale,
                                      tra_stream_t stream) {
+  NvtxRange nvtx_range("tra_block_sparse_attn_fp8");
   tra_status s = check_attn_common(Q8, K8, V, O, heads, N, d, scale);
   if (s != TRA_OK) return s;
   if (d != 128 || block_q != 128 || block_k != 128) return TRA_ERR_UNSUPPORTED;
@@ -239,6 +255,7 @@ tra_status tra_block_sparse_attn_fp8(const void* Q8, const float* q_scales, cons
 tra_status tra_budget_radius_ex(const float* H, float* r, float* phi_out, int heads,
                                 tra_grid grid, tra_tile tile, float tau, float gamma,
                                 tra_budget budget, tra_metric metric, tra_stream_t stream) {
+  NvtxRange nvtx_range("tra_budget_radius_ex");
   if (heads < 0 || !grid_ok(grid) || !tile_ok(tile)) return TRA_ERR_INVALID_ARGUMENT;
   if (!(tau >= 0.f) || !std::isfinite(tau) || !(gamma >= 0.f) || !std::isfinite(gamma))
     return TRA_ERR_INVALID_ARGUMENT;
@@ -299,6 +316,7 @@ tra_status tra_budget_radius(const float* H, float* r, float* phi_out, int heads
 
 tra_status tra_radial_radius(float* r, float* phi_out, int heads, tra_grid grid, tra_tile tile,
                              float r0, tra_metric metric, tra_stream_t stream) {
+  NvtxRange nvtx_range("tra_radial_radius");
   if (heads < 0 || !grid_ok(grid) || !tile_ok(tile)) return TRA_ERR_INVALID_ARGUMENT;
   if (!(r0 >= 0.f)) return TRA_ERR_INVALID_ARGUMENT;  // NaN and negative radii
   if (metric != TRA_METRIC_DISK && metric != TRA_METRIC_LINE) return TRA_ERR_INVALID_ARGUMENT;
@@ -335,6 +353,7 @@ tra_status tra_build_block_mask_ex(const float* r, const float* phi, int heads, 
                                    tra_metric metric, int* row_ptr, int* col_idx,
                                    long long col_capacity, int* nnz, void* workspace,
                                    size_t workspace_bytes, tra_stream_t stream) {
+  NvtxRange nvtx_range("tra_build_block_mask_ex");
   if (heads < 0 || !grid_ok(grid) || !tile_ok(tile)) return TRA_ERR_INVALID_ARGUMENT;
   if (metric != TRA_METRIC_DISK && metric != TRA_METRIC_LINE) return TRA_ERR_INVALID_ARGUMENT;
   if (!block_ok(block_q) || !block_ok(block_k)) return TRA_ERR_UNSUPPORTED;
@@ -375,6 +394,15 @@ tra_status tra_build_block_mask(const float* r, const float* phi, int heads, tra
   return tra_build_block_mask_ex(r, phi, heads, grid, tile, block_q, block_k, vote_threshold,
                                  TRA_METRIC_DISK, row_ptr, col_idx, col_capacity, nnz, workspace,
                                  workspace_bytes, stream);
+}
+
+tra_status tra_selftest_wait_timeout(int limit_ms, int* completed, tra_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return TRA_ERR_INVALID_ARGUMENT;
+  if (completed != nullptr && !aligned16(completed)) return TRA_ERR_INVALID_ARGUMENT;
+  const tra_status dv = check_device();
+  if (dv != TRA_OK) return dv;
+  return status_of(launch_selftest_wait(static_cast<unsigned long long>(limit_ms) * 1000000ull,
+                                        completed, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tra_status tra_get_device_error(int* code, tra_stream_t stream) {

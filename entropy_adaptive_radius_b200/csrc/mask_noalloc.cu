@@ -21,10 +21,17 @@
 #include <cstdint>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "tra_internal.h"
 
 namespace tra {
 namespace {
+
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 constexpr size_t kMaskStaticScratchBytes = static_cast<size_t>(TRA_MASK_STATIC_SCRATCH_BYTES);
 
@@ -66,6 +73,7 @@ extern "C" tra_status tra_build_block_mask_noalloc(const float* r, const float* 
                                                    int* col_idx, long long col_capacity,
                                                    int* nnz, tra_stream_t stream) {
   using namespace tra;
+  NvtxRange nvtx_range("tra_build_block_mask_noalloc");
   if (heads < 0 || grid.F < 0 || grid.H < 0 || grid.W < 0 || grid.F > kMaxFrames ||
       grid.H > kMaxSide || grid.W > kMaxSide ||
       static_cast<long long>(grid.F) * grid.H * grid.W > (1LL << 24) || tile.t < 1 ||

@@ -24,6 +24,7 @@ enum DeviceError : int {
   kErrWaitPFull = 8,
   kErrWaitPVDone = 9,
   kErrBadCsr = 10,
+  kErrSelfTest = 11,  // the self-test's wait on a barrier nothing completes
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -103,13 +104,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // case it sets *abort and records `code` in the device error word.
 // Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* err, int code) {
+                                          int* err, int code,
+                                          unsigned long long limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait_sleep(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait_sleep(bar, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *abort = 1;
       if (err) atomicCAS(err, 0, code);
       return false;

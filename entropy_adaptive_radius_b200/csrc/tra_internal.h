@@ -68,6 +68,8 @@ struct AttnArgs {
   const float* q_scales;  // [heads, ceil(N / 128)] (fp8 only)
   const float* k_scales;  // [heads, ceil(N / 128)] (fp8 only)
 };
+// selftest.cu: one wait on a barrier nothing completes, given up after limit_ns
+cudaError_t launch_selftest_wait(unsigned long long limit_ns, int* completed, cudaStream_t stream);
 // quant.cu: per (head, block of `block` rows) E4M3 quantization of bf16 X
 cudaError_t launch_quantize_e4m3(const void* X, void* Xq, float* scales, int heads, int N, int d,
                                  int block, cudaStream_t stream);

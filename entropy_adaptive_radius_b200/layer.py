@@ -111,6 +111,37 @@ class TraLayer:
         """Start a new denoising run (the next step is a warm-up step again)."""
         self.step_index = 0
 
+    def _meta(self):
+        return {"grid": list(self.grid), "heads": self.heads, "d": self.d, "tile": list(self.tile),
+                "block_q": self.block_q, "block_k": self.block_k, "tau": self.tau,
+                "gamma": self.gamma, "vote": self.vote, "budget": self.budget,
+                "metric": self.metric, "radial_r0": self.radial_r0}
+
+    def state_dict(self) -> dict:
+        """What the following steps reuse: the entropy of the last refresh, the
+        radii, the decay table, the CSR mask and the step index (copies, on the
+        layer's device), with the settings they were built under.  Save it with
+        torch.save to resume a denoising run without a new warm-up."""
+        nnz = int(self.nnz.item())
+        return {"meta": self._meta(), "step_index": self.step_index, "H": self.H.clone(),
+                "r": self.r.clone(), "phi": self.phi.clone(), "row_ptr": self.row_ptr.clone(),
+                "col_idx": self.col_idx[:nnz].clone(), "nnz": nnz}
+
+    def load_state_dict(self, state: dict):
+        """Restore a state_dict taken from a layer with the same settings."""
+        if state["meta"] != self._meta():
+            raise ValueError("state was taken from a layer with other settings")
+        nnz = int(state["nnz"])
+        if nnz > self.col_idx.numel() or state["row_ptr"].numel() != self.row_ptr.numel():
+            raise ValueError("state does not fit this layer's mask buffers")
+        self.H.copy_(state["H"])
+        self.r.copy_(state["r"])
+        self.phi.copy_(state["phi"])
+        self.row_ptr.copy_(state["row_ptr"])
+        self.col_idx[:nnz].copy_(state["col_idx"])
+        self.nnz.fill_(nnz)
+        self.step_index = int(state["step_index"])
+
     def _rebuild_mask(self):
         if self.radial_r0 is not None:
             tra.tra_radial_radius(self.r, self.grid, self.radial_r0, self.metric, self.tile,

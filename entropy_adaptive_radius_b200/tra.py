@@ -69,6 +69,7 @@ _PROTOS = {
     "tra_quantize_e4m3": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp]),
     "tra_block_sparse_attn_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int,
                                            _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
+    "tra_selftest_wait_timeout": (_c_int, [_c_int, _vp, _vp]),
     "tra_get_device_error": (_c_int, [ctypes.POINTER(_c_int), _vp]),
 }
 
@@ -284,6 +285,14 @@ def tra_block_sparse_attn_fp8(Q8, q_scales, K8, k_scales, V, O, row_ptr, col_idx
         _p(Q8), _p(q_scales), _p(K8), _p(k_scales), _p(V), _p(O), _p(lse), _p(row_ptr),
         _p(col_idx), heads, N, d, block_q, block_k, scale, _stream(stream)))
     return O
+
+
+def tra_selftest_wait_timeout(limit_ms, completed=None, stream=None):
+    """Launch the bounded-wait self-test (a wait that nothing completes, given
+    up after limit_ms); read the outcome with tra_get_device_error."""
+    _contig(completed)
+    _check("tra_selftest_wait_timeout", lib().tra_selftest_wait_timeout(
+        int(limit_ms), _p(completed), _stream(stream)))
 
 
 def tra_get_device_error(stream=None) -> int:

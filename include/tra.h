@@ -345,6 +345,19 @@ tra_status tra_block_sparse_attn_fp8(const void* Q8, const float* q_scales, cons
                                      tra_stream_t stream);
 
 /*
+ * Self-test of failure detection.  Launches one kernel that waits, with the
+ * same bounded-wait helper every kernel here uses, on a barrier that nothing
+ * ever completes.  After `limit_ms` the wait gives up, the kernel records
+ * code 11 in the device error word and returns, so the context stays usable:
+ * the next tra_get_device_error returns TRA_ERR_TIMEOUT with *code = 11.
+ *   limit_ms   1 .. 2000.
+ *   completed  [1] int32 device pointer (16-byte aligned) or NULL; written:
+ *              1 if the wait completed (it never should), 0 if it gave up.
+ * The other kernels use a limit of 4 s.
+ */
+tra_status tra_selftest_wait_timeout(int limit_ms, int* completed, tra_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word of the
  * current device.  *code = 0 when no kernel recorded an error; otherwise the
  * code of the first wait that ran out of time.  Returns TRA_ERR_TIMEOUT when

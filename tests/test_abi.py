@@ -171,3 +171,10 @@ def test_fp8_validation(L):
     assert a(P, None, P, P, P, P, None, P, P, 2, 1000, 128, 128, 128, 0.1, S0) == INVALID
     assert a(P, P, P, P, P, P, None, None, P, 2, 1000, 128, 128, 128, 0.1, S0) == INVALID
     assert a(P, P, P, P, P, P, None, P, P, 2, 1000, 128, 128, 128, 0.0, S0) == INVALID
+
+
+def test_selftest_validation(L):
+    st = L.tra_selftest_wait_timeout
+    assert st(0, None, S0) == INVALID
+    assert st(3000, None, S0) == INVALID
+    assert st(10, MIS, S0) == INVALID

@@ -1,0 +1,72 @@
+"""Failure detection and resumable state on the GPU.
+
+The bounded-wait self-test waits on a barrier nothing completes: the wait
+must give up after its limit, report TRA_ERR_TIMEOUT with its code, clear on
+reading, and leave the context usable.  A layer's reuse state (entropy,
+radii, mask, step index) saved after the warm-up and loaded into a fresh
+layer must reproduce the original layer's next steps bit for bit."""
+import io
+import math
+import time
+
+import numpy as np
+import pytest
+import torch
+
+from entropy_adaptive_radius_b200 import inputs, tra
+from entropy_adaptive_radius_b200.layer import ReusePolicy, TraLayer
+from oracle import tra_oracle as O
+from tests.gpu_util import check_attention, need_gpu, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_gives_up_reports_and_context_survives():
+    need_gpu()
+    assert tra.tra_get_device_error() == 0
+    flag = torch.full((4,), 7, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.time()
+    tra.tra_selftest_wait_timeout(50, flag)
+    code = tra.tra_get_device_error()        # synchronises the stream
+    dt = time.time() - t0
+    assert code == 11
+    assert int(flag[0].item()) == 0          # the wait gave up, it did not complete
+    assert 0.045 < dt < 2.0
+    assert tra.tra_get_device_error() == 0   # the word is cleared by reading it
+    # the context still runs the attention kernels correctly
+    g = torch.Generator().manual_seed(4)
+    Q, K, V = (torch.randn(1, 300, 64, generator=g).to(torch.bfloat16) for _ in range(3))
+    O_ = torch.empty(1, 300, 64, dtype=torch.bfloat16, device="cuda")
+    H = torch.empty(1, 300, dtype=torch.float32, device="cuda")
+    tra.tra_dense_attn_entropy(Q.cuda(), K.cuda(), V.cuda(), O_, H)
+    assert tra.tra_get_device_error() == 0
+    Or, _, _ = O.dense_attention_entropy(to64(Q), to64(K), to64(V), 1.0 / math.sqrt(64))
+    check_attention(O_, Or, "O after the timeout")
+
+
+def test_layer_state_round_trip_resumes_bit_for_bit():
+    need_gpu()
+    grid, heads, d = (4, 12, 16), 2, 64
+    N = 4 * 12 * 16
+    policy = ReusePolicy(warmup=1, refresh_every=3, refresh="entropy")
+    kw = dict(tau=0.2, gamma=0.3, block_q=64, block_k=64, policy=policy)
+    Q, K, V = inputs.make_qkv(*grid, heads, d, 7, (0.5, 4.0), "bf16")
+    steps = [(inputs.perturb(Q, 7, c, 0), inputs.perturb(K, 7, c, 1), V) for c in range(1, 6)]
+    a = TraLayer(grid, heads, d, **kw)
+    a(Q.cuda(), K.cuda(), V.cuda())                      # warm-up: entropy and mask
+    buf = io.BytesIO()
+    torch.save(a.state_dict(), buf)
+    buf.seek(0)
+    b = TraLayer(grid, heads, d, **kw)
+    b.load_state_dict(torch.load(buf))
+    assert b.step_index == a.step_index == 1
+    for q, k, v in steps:                                 # sparse steps and a refresh
+        Oa = a(q.cuda(), k.cuda(), v.cuda())
+        Ob = b(q.cuda(), k.cuda(), v.cuda())
+        assert torch.equal(Oa, Ob)
+        assert torch.equal(a.row_ptr, b.row_ptr)
+    assert tra.tra_get_device_error() == 0
+    c = TraLayer(grid, heads, d, tau=0.3, gamma=0.3, block_q=64, block_k=64, policy=policy)
+    with pytest.raises(ValueError):
+        c.load_state_dict(a.state_dict())
