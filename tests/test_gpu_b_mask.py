@@ -166,3 +166,24 @@ def test_mask_full_size_sampled(wl, vote):
                         assert qb in set(csr_rows(rp, ci, h, qb, nqb).tolist())
     kept = nnz / (wl.heads * nqb * nkb)
     assert 0.0 < kept < 1.0
+
+
+@pytest.mark.parametrize("grid,tile,bq,bk,vote", [((1, 9, 13), (1, 4, 4), 16, 16, 1),
+                                                  ((384, 4, 4), (1, 4, 4), 16, 16, 20),
+                                                  ((384, 4, 4), (2, 4, 4), 64, 16, 70)])
+def test_mask_frame_count_extremes(grid, tile, bq, bk, vote):
+    """One frame, and the largest frame count the mask accepts (its per-frame
+    threshold table then needs the opt-in shared-memory size).  Every query
+    keeps its own (x, y) in every frame, so with many small frames the vote
+    threshold is set above those self votes to make the mask non-trivial."""
+    need_gpu()
+    F, H, W = grid
+    N = F * H * W
+    r = inputs.synthetic_radius(2, N, seed=F + bq, lo=0.3, hi=3.0, special=False)
+    phi = O.phi(np.arange(F), 0.6).astype(np.float32)
+    rp, ci, nnz = run_mask(r, phi, grid, tile, bq, bk, vote)
+    rp_ref, ci_ref, _ = oracle_csr(r, phi, grid, tile, bq, bk, vote)
+    assert nnz == len(ci_ref)
+    assert np.array_equal(rp, rp_ref)
+    assert np.array_equal(ci[:nnz], ci_ref)
+    assert 0.0 < nnz / (2 * (-(-N // bq)) * (-(-N // bk))) < 1.0
