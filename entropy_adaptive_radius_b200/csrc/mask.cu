@@ -36,7 +36,8 @@
 namespace tra {
 namespace {
 
-constexpr int kMaxSeg = 4;  // per-frame boxes kept per key block (more: no pruning)
+constexpr int kMaxSeg = 4;   // per-frame boxes kept per key block (more: no pruning)
+constexpr int kMaxRect = 4;  // complete rectangles kept per key block (more: row tests)
 constexpr int kVoteThreads = 128;
 constexpr int kRsqCap = 1 << 30;
 constexpr int kReachCap = 1 << 30;  // 1D reach cap: beyond any in-frame index distance (< 2^24)
@@ -45,6 +46,7 @@ struct MaskWs {
   uint2* rows;      // [nkb * Bk]: x = t << 16 | y, y = x_lo << 16 | x_hi
   int4* info;       // [nkb]: x = rows (-1: not row-contiguous), y = segments (-1: too many), z = tokens
   int4* segs;       // [nkb * kMaxSeg]: x = t, y = y_lo << 16 | y_hi, z = x_lo << 16 | x_hi
+  int4* rects;      // [nkb * kMaxRect]: as segs, every position of the rectangle a key of the block
   uint32_t* bits;   // [heads * nqb * nkbw]
   int* counts;      // [heads * nqb]
 };
@@ -70,16 +72,19 @@ size_t carve(const TileLayout& L, int heads, int bq, int bk, char* base, MaskWs*
   const size_t rows = align256(sizeof(uint2) * static_cast<size_t>(m.nkb) * bk);
   const size_t info = align256(sizeof(int4) * static_cast<size_t>(m.nkb));
   const size_t segs = align256(sizeof(int4) * static_cast<size_t>(m.nkb) * kMaxSeg);
+  const size_t rects = align256(sizeof(int4) * static_cast<size_t>(m.nkb) * kMaxRect);
   const size_t bits = align256(sizeof(uint32_t) * static_cast<size_t>(heads) * m.nqb * m.nkbw);
   const size_t counts = align256(sizeof(int) * static_cast<size_t>(heads) * m.nqb);
   if (ws) {
-    ws->rows = reinterpret_cast<uint2*>(base + off);
-    ws->info = reinterpret_cast<int4*>(base + off + rows);
-    ws->segs = reinterpret_cast<int4*>(base + off + rows + info);
-    ws->bits = reinterpret_cast<uint32_t*>(base + off + rows + info + segs);
-    ws->counts = reinterpret_cast<int*>(base + off + rows + info + segs + bits);
+    char* q = base + off;
+    ws->rows = reinterpret_cast<uint2*>(q);
+    ws->info = reinterpret_cast<int4*>(q += rows);
+    ws->segs = reinterpret_cast<int4*>(q += info);
+    ws->rects = reinterpret_cast<int4*>(q += segs);
+    ws->bits = reinterpret_cast<uint32_t*>(q += rects);
+    ws->counts = reinterpret_cast<int*>(q += bits);
   }
-  return rows + info + segs + bits + counts;
+  return rows + info + segs + rects + bits + counts;
 }
 
 __device__ __forceinline__ int isqrt_floor(int m) {
@@ -165,7 +170,37 @@ __global__ void footprint_kernel(TileLayout L, int bk, MaskWs ws) {
   const int tokens = p1 - p0;
   for (int i = 0; i < max(nseg, 0); ++i)
     segs[i] = make_int4(st[i], (sylo[i] << 16) | syhi[i], (sxlo[i] << 16) | sxhi[i], 0);
-  ws.info[kb] = make_int4(span == tokens ? nrows : -1, nseg, tokens, 0);
+  // Complete rectangles: consecutive rows of one frame with consecutive y and
+  // the same x interval.  With contiguous rows every position of such a
+  // rectangle is a key of the block, so a disk meets a key of the block iff
+  // it meets one of the rectangles.
+  int nrect = -1;
+  if (span == tokens) {
+    int4* rects = ws.rects + static_cast<size_t>(kb) * kMaxRect;
+    nrect = 0;
+    int ct = -1, cylo = 0, cyhi = 0, cx = 0;
+    for (int i = 0; i <= nrows && nrect >= 0; ++i) {
+      int t = -1, y = 0, xr = 0;
+      if (i < nrows) {
+        t = static_cast<int>(rows[i].x >> 16);
+        y = static_cast<int>(rows[i].x & 0xFFFFu);
+        xr = static_cast<int>(rows[i].y);
+        if (t == ct && y == cyhi + 1 && xr == cx) {
+          cyhi = y;
+          continue;
+        }
+      }
+      if (ct >= 0) {  // close the current rectangle
+        if (nrect == kMaxRect) {
+          nrect = -1;
+          break;
+        }
+        rects[nrect++] = make_int4(ct, (cylo << 16) | cyhi, cx, 0);
+      }
+      ct = t; cylo = cyhi = y; cx = xr;
+    }
+  }
+  ws.info[kb] = make_int4(span == tokens ? nrows : -1, nseg, tokens, nrect);
 }
 
 // -------------------------------------------------------------------- 2. votes
@@ -305,7 +340,60 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
       cand &= cand - 1;
       const int kb2 = w * 32 + b;
       const int nrows = __shfl_sync(0xffffffffu, info.x, b);
+      const int nseg = __shfl_sync(0xffffffffu, info.y, b);
+      const int nrect = __shfl_sync(0xffffffffu, info.w, b);
       bool keep = false;
+      if constexpr (!LINE) {
+        // vote threshold 1 and complete rectangles: the disk / rectangle test
+        // is exact (the nearest lattice point of a rectangle to the query is
+        // one of its keys), so it decides the block without row tests
+        if (exists && nrect >= 0) {
+          const int4* rc = ws.rects + static_cast<size_t>(kb2) * kMaxRect;
+          bool hit = false;
+          for (int i = 0; i < nrect; ++i) {
+            const int4 rr = rc[i];
+            const int* rs = s_rsq + rr.x * 128 + lane;
+            const int ylo = rr.y >> 16, yhi = rr.y & 0xFFFF;
+            const int xlo = rr.z >> 16, xhi = rr.z & 0xFFFF;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int lim = rs[32 * k];
+              const int dx = max(0, max(xlo - qx[k], qx[k] - xhi));
+              const int dy = max(0, max(ylo - qy[k], qy[k] - yhi));
+              hit |= (lim >= 0) & (dx * dx + dy * dy <= lim);
+            }
+          }
+          if (__any_sync(0xffffffffu, hit)) word |= 1u << b;
+          continue;
+        }
+      }
+      // Exact rejection first: if no query's disk (interval) meets any of the
+      // block's per-frame boxes, no key of the block is inside any support.
+      // One test per (query, box) instead of one per (query, row).
+      if (nseg > 0) {
+        const int4* sg = ws.segs + static_cast<size_t>(kb2) * kMaxSeg;
+        bool hit = false;
+        for (int i = 0; i < nseg; ++i) {
+          const int4 sgm = sg[i];
+          const int* rs = s_rsq + sgm.x * 128 + lane;
+          const int ylo = sgm.y >> 16, yhi = sgm.y & 0xFFFF;
+          const int xlo = sgm.z >> 16, xhi = sgm.z & 0xFFFF;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int lim = rs[32 * k];
+            if constexpr (LINE) {
+              const int nlo = ylo * L.W + xlo, nhi = yhi * L.W + xhi;
+              const int dn = max(0, max(nlo - qx[k], qx[k] - nhi));
+              hit |= (lim >= 0) & (dn <= lim);
+            } else {
+              const int dx = max(0, max(xlo - qx[k], qx[k] - xhi));
+              const int dy = max(0, max(ylo - qy[k], qy[k] - yhi));
+              hit |= (lim >= 0) & (dx * dx + dy * dy <= lim);
+            }
+          }
+        }
+        if (!__any_sync(0xffffffffu, hit)) continue;  // not kept: no votes at all
+      }
       if (nrows >= 0) {
         const uint2* rows = ws.rows + static_cast<size_t>(kb2) * bk;
         int votes = 0;
