@@ -286,17 +286,26 @@ def time_ms(fn, reps=5):
     return statistics.median(ts)
 
 
+def code_sha256(path):
+    """sha256 of a C++/CUDA source with comments and whitespace removed: it
+    changes when the code changes, not when only its comments do."""
+    import hashlib
+    import re
+    src = open(path).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return hashlib.sha256(re.sub(r"\s+", " ", src).strip().encode()).hexdigest()
+
+
 def measured_traffic(wl, kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu capture of this
-    workload, or None when there is none or the kernel source has changed
-    since it was taken."""
-    import hashlib
+    workload, or None when there is none or the kernel code has changed since
+    it was taken."""
     path = os.path.join(ROOT, "profiles", "dram_traffic_wan14b.txt")
     if wl.name != workloads.WAN14B.name or not os.path.exists(path):
         return None
     rec = json.load(open(path))
-    src = open(os.path.join(ROOT, rec["source"]), "rb").read()
-    if hashlib.sha256(src).hexdigest() != rec["source_sha256"] or kernel not in rec:
+    if code_sha256(os.path.join(ROOT, rec["source"])) != rec["source_code_sha256"] or kernel not in rec:
         return None
     return rec[kernel]["traffic_bytes"]
 

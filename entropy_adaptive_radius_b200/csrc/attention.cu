@@ -6,21 +6,26 @@
 // (fused entropy kernel), efficient execution (block-sparse attention over the
 // kept query-block x key-block pairs, reused across sparse steps).
 //
-// One CTA computes 128 query rows of one head against a list of key blocks
-// (all blocks for the dense pass; the CSR row for the sparse pass; when
-// query blocks are smaller than 128 rows, the union of the rows' lists with
-// per-row masking).  Warp roles:
-//   warp 0      TMA producer: Q once, then K and V tiles into a 2-stage ring
-//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
-//               score buffers, O += P_j V_j into a TMEM accumulator
-//   warp 2      allocates / frees tensor memory
-//   warps 4..7  softmax: thread i owns query row i (TMEM lane i); reads S_j,
-//               keeps the running max m, Z = sum 2^(u-m) and
-//               A = sum 2^(u-m) (u-m) (u = s*log2 e), writes P_j (bf16) to
-//               shared memory in the MMA's swizzled layout, rescales O when
-//               the max grows by more than 2^8, and writes O / Z, the entropy
-//               H = ln Z - ln 2 * A / Z and LSE = ln 2 * (m + log2 Z).
-// S_{j+1} runs on the tensor cores while the softmax of block j runs.
+// Three kernels, each with one CTA per (128-row query tile, head):
+//   attn_dual_kernel  the dense pass and block-sparse attention with 64- or
+//                     128-token blocks: two softmax warpgroups split the key
+//                     blocks, separate K / V producers and QK / PV issuers
+//                     (described at the kernel);
+//   attn_kernel       block-sparse attention when a block is 16 tokens (up to
+//                     eight query blocks per tile, their lists merged in shared
+//                     memory): one softmax warpgroup;
+//   entropy_kernel    the entropy-only pass (no PV, no output).
+// In all of them thread i of a softmax warpgroup owns query row i (TMEM lane
+// i): it reads the score tile S_j, keeps the running max m, Z = sum 2^(u-m)
+// and A = sum 2^(u-m) (u-m) (u = s * log2 e), writes P_j (bf16) to shared
+// memory in the MMA's swizzled layout, rescales O when the max grows by more
+// than 2^8, and finally writes O / Z, the entropy H = ln Z - ln 2 * A / Z and
+// LSE = ln 2 * (m + log2 Z).  The tensor cores compute the next score tile
+// while the softmax of the current one runs.
+//
+// attn_kernel's warp roles: warp 0 TMA producer (Q once, then K and V into a
+// 2-stage ring), warp 1 MMA issuer (S_j into one of two TMEM score buffers,
+// O += P_j V_j), warp 2 tensor-memory allocation, warps 4..7 softmax.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
@@ -582,7 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Two-warpgroup variant for 128-row query blocks and 128-key blocks.
+// Two-warpgroup kernel: the dense pass and block-sparse attention with 64- or
+// 128-token blocks (16-token blocks use attn_kernel above).
 //
 // The CTA owns one 128-row query tile.  Its key-block list is split between
 // two softmax warpgroups: warpgroup w (warps 4w .. 4w+3) takes blocks
@@ -590,9 +596,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // accumulator O_w, its own bf16 P_w buffer in shared memory and its own
 // running statistics (m_w, Z_w, A_w).  Each warpgroup therefore has two block
 // periods of tensor-core work to hide one softmax iteration, and each
-// scheduler has two softmax warps to issue from.  The MMA warp issues QK^T two
-// blocks ahead of PV (S_{j+2} as soon as warpgroup j mod 2 has read S_j), so a
-// score tile is ready when its warpgroup finishes the previous one.  K and V
+// scheduler has two softmax warps to issue from.  QK^T runs two blocks ahead
+// of PV (S_{j+2} as soon as warpgroup j mod 2 has read S_j), so a score tile
+// is ready when its warpgroup finishes the previous one.  K and V
 // have separate producer warps so that prefetching K never waits behind a V
 // slot that is still in use.  At the end the two partial results are merged
 // exactly:

@@ -45,14 +45,13 @@ def test_measured_traffic_needs_the_captured_source(tmp_path, monkeypatch):
     wl = workloads.WAN14B
     got = bench.measured_traffic(wl, "dense_attn_entropy")
     src = open(os.path.join(bench.ROOT, rec["source"]), "rb").read()
-    import hashlib
-    if hashlib.sha256(src).hexdigest() == rec["source_sha256"]:
+    if bench.code_sha256(os.path.join(bench.ROOT, rec["source"])) == rec["source_code_sha256"]:
         assert got == rec["dense_attn_entropy"]["traffic_bytes"]
     else:
         assert got is None
-    # another workload, or a changed source, gives no figure
+    # another workload, or changed code, gives no figure
     assert bench.measured_traffic(workloads.WAN13B, "dense_attn_entropy") is None
-    fake = dict(rec, source_sha256="0" * 64)
+    fake = dict(rec, source_code_sha256="0" * 64)
     p = tmp_path / "profiles"
     p.mkdir()
     (p / "dram_traffic_wan14b.txt").write_text(json.dumps(fake))
@@ -71,3 +70,14 @@ def test_traffic_record_is_near_the_algorithmic_bytes():
         r = rec[k]
         assert r["traffic_bytes"] == r["dram_read_bytes"] + r["dram_write_bytes"]
         assert 0.95 < r["traffic_bytes"] / r["algorithmic_bytes"] < 1.1
+
+
+def test_code_hash_ignores_comments_only(tmp_path):
+    a = tmp_path / "a.cu"
+    b = tmp_path / "b.cu"
+    c = tmp_path / "c.cu"
+    a.write_text("int f(int x) {  // twice\n  return 2 * x; }\n")
+    b.write_text("/* doubles */\nint f(int x) {\n  return 2 * x;\n}\n")
+    c.write_text("int f(int x) { return 3 * x; }\n")
+    assert bench.code_sha256(str(a)) == bench.code_sha256(str(b))
+    assert bench.code_sha256(str(a)) != bench.code_sha256(str(c))
