@@ -14,12 +14,8 @@
 
 namespace tra {
 
-// One NVTX range per API call (named after the call), visible to Nsight
-// tools; with no tool attached the calls do nothing.
-struct NvtxRange {
-  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
-  ~NvtxRange() { nvtxRangePop(); }
-};
+NvtxRange::NvtxRange(const char* name) { nvtxRangePushA(name); }
+NvtxRange::~NvtxRange() { nvtxRangePop(); }
 
 // Device error word: first code recorded by a kernel whose wait ran out of time.
 __device__ int g_device_error = 0;
@@ -33,27 +29,42 @@ int g_cc_ok[kMaxDevices] = {};  // 0 unknown, 1 sm_100, -1 other
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-tra_status check_device() {
+tra_status status_of(cudaError_t e) {
+  if (e == cudaSuccess) return TRA_OK;
+  return TRA_ERR_CUDA;
+}
+
+}  // namespace
+
+tra_status check_device(std::initializer_list<const void*> ptrs) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
     return TRA_ERR_DEVICE;
   }
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (g_cc_ok[dev] == 0) {
-    int major = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
-      cudaGetLastError();
-      return TRA_ERR_DEVICE;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_cc_ok[dev] == 0) {
+      int major = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return TRA_ERR_DEVICE;
+      }
+      g_cc_ok[dev] = (major == 10) ? 1 : -1;
     }
-    g_cc_ok[dev] = (major == 10) ? 1 : -1;
+    if (g_cc_ok[dev] != 1) return TRA_ERR_DEVICE;
   }
-  return g_cc_ok[dev] == 1 ? TRA_OK : TRA_ERR_DEVICE;
-}
-
-tra_status status_of(cudaError_t e) {
-  if (e == cudaSuccess) return TRA_OK;
-  return TRA_ERR_CUDA;
+  for (const void* p : ptrs) {
+    if (p == nullptr) continue;
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+      cudaGetLastError();
+      return TRA_ERR_INVALID_ARGUMENT;
+    }
+    if (at.type == cudaMemoryTypeManaged) continue;
+    if (at.type != cudaMemoryTypeDevice || at.device != dev) return TRA_ERR_INVALID_ARGUMENT;
+  }
+  return TRA_OK;
 }
 
 bool grid_ok(const tra_grid& g) {
@@ -68,8 +79,6 @@ bool block_ok(int b) { return b == 16 || b == 64 || b == 128; }
 TileLayout layout_of(const tra_grid& g, const tra_tile& t) {
   return TileLayout{g.F, g.H, g.W, t.t, t.y, t.x};
 }
-
-}  // namespace
 
 int* device_error_word() {
   int dev = 0;
@@ -95,7 +104,7 @@ extern "C" {
 const char* tra_status_string(tra_status s) {
   switch (s) {
     case TRA_OK: return "ok";
-    case TRA_ERR_INVALID_ARGUMENT: return "invalid argument (null pointer, bad size or misaligned pointer)";
+    case TRA_ERR_INVALID_ARGUMENT: return "invalid argument (null, misaligned or host pointer, or bad size)";
     case TRA_ERR_UNSUPPORTED: return "unsupported shape (d, block size or list length)";
     case TRA_ERR_WORKSPACE: return "workspace too small or not 256-byte aligned";
     case TRA_ERR_CAPACITY: return "negative col_idx capacity";
@@ -122,7 +131,7 @@ tra_status tra_tile_major_permute(const void* X, void* X_tm, tra_dtype in_dtype,
   if (X == nullptr || X_tm == nullptr || !aligned16(X) || !aligned16(X_tm))
     return TRA_ERR_INVALID_ARGUMENT;
   if (X == X_tm) return TRA_ERR_INVALID_ARGUMENT;
-  const tra_status dv = check_device();
+  const tra_status dv = check_device({X, X_tm});
   if (dv != TRA_OK) return dv;
   return status_of(launch_permute(X, X_tm, in_dtype, out_dtype, heads, d, layout_of(grid, tile),
                                   false, reinterpret_cast<cudaStream_t>(stream)));
@@ -140,7 +149,7 @@ tra_status tra_inverse_permute(const void* X_tm, void* X, tra_dtype dtype, int h
   if (X == nullptr || X_tm == nullptr || !aligned16(X) || !aligned16(X_tm))
     return TRA_ERR_INVALID_ARGUMENT;
   if (X == X_tm) return TRA_ERR_INVALID_ARGUMENT;
-  const tra_status dv = check_device();
+  const tra_status dv = check_device({X, X_tm});
   if (dv != TRA_OK) return dv;
   return status_of(launch_permute(X_tm, X, dtype, dtype, heads, d, layout_of(grid, tile), true,
                                   reinterpret_cast<cudaStream_t>(stream)));
@@ -166,7 +175,7 @@ tra_status tra_dense_attn_entropy(const void* Q, const void* K, const void* V, v
   tra_status s = check_attn_common(Q, K, V, O, heads, N, d, scale);
   if (s != TRA_OK || heads == 0 || N == 0) return s;
   if (H == nullptr) return TRA_ERR_INVALID_ARGUMENT;
-  s = check_device();
+  s = check_device({Q, K, V, O, H, lse});
   if (s != TRA_OK) return s;
   AttnArgs a{};
   a.Q = Q; a.K = K; a.V = V; a.O = O; a.H = H; a.lse = lse;
@@ -184,7 +193,7 @@ tra_status tra_attn_entropy(const void* Q, const void* K, float* H, float* lse, 
   if (heads == 0 || N == 0) return TRA_OK;
   if (heads > 65535 || N > (1 << 24)) return TRA_ERR_UNSUPPORTED;
   if (!Q || !K || !H || !aligned16(Q) || !aligned16(K)) return TRA_ERR_INVALID_ARGUMENT;
-  const tra_status s = check_device();
+  const tra_status s = check_device({Q, K, H, lse});
   if (s != TRA_OK) return s;
   AttnArgs a{};
   a.Q = Q; a.K = K; a.V = nullptr; a.O = nullptr; a.H = H; a.lse = lse;
@@ -206,7 +215,7 @@ tra_status tra_block_sparse_attn(const void* Q, const void* K, const void* V, vo
   // 16-token blocks run on the kernel that merges up to eight query blocks'
   // lists in shared memory (at most 1024 key blocks)
   if (block_q < 128 && (block_q == 16 || block_k == 16) && nkb > 1024) return TRA_ERR_UNSUPPORTED;
-  s = check_device();
+  s = check_device({Q, K, V, O, lse, row_ptr, col_idx});
   if (s != TRA_OK) return s;
   AttnArgs a{};
   a.Q = Q; a.K = K; a.V = V; a.O = O; a.H = nullptr; a.lse = lse;
@@ -224,7 +233,7 @@ tra_status tra_quantize_e4m3(const void* X, void* Xq, float* scales, int heads, 
   if (heads == 0 || N == 0) return TRA_OK;
   if (heads > 65535 || N > (1 << 24)) return TRA_ERR_UNSUPPORTED;
   if (!X || !Xq || !scales || !aligned16(X) || !aligned16(Xq)) return TRA_ERR_INVALID_ARGUMENT;
-  const tra_status dv = check_device();
+  const tra_status dv = check_device({X, Xq, scales});
   if (dv != TRA_OK) return dv;
   return status_of(launch_quantize_e4m3(X, Xq, scales, heads, N, d, block,
                                         reinterpret_cast<cudaStream_t>(stream)));
@@ -241,7 +250,7 @@ tra_status tra_block_sparse_attn_fp8(const void* Q8, const float* q_scales, cons
   if (d != 128 || block_q != 128 || block_k != 128) return TRA_ERR_UNSUPPORTED;
   if (heads == 0 || N == 0) return TRA_OK;
   if (!row_ptr || !col_idx || !q_scales || !k_scales) return TRA_ERR_INVALID_ARGUMENT;
-  s = check_device();
+  s = check_device({Q8, q_scales, K8, k_scales, V, O, lse, row_ptr, col_idx});
   if (s != TRA_OK) return s;
   AttnArgs a{};
   a.Q = Q8; a.K = K8; a.V = V; a.O = O; a.H = nullptr; a.lse = lse;
@@ -266,7 +275,7 @@ tra_status tra_budget_radius_ex(const float* H, float* r, float* phi_out, int he
   if (heads == 0 && phi_out == nullptr) return TRA_OK;
   if (heads > 0 && (H == nullptr || r == nullptr)) return TRA_ERR_INVALID_ARGUMENT;
   if (heads > 65535) return TRA_ERR_UNSUPPORTED;
-  const tra_status dv = check_device();
+  const tra_status dv = check_device({H, r, phi_out});
   if (dv != TRA_OK) return dv;
   const bool line = metric == TRA_METRIC_LINE;
   // phi(delta) = exp(-gamma delta); per query frame t the disk uses
@@ -325,7 +334,7 @@ tra_status tra_radial_radius(float* r, float* phi_out, int heads, tra_grid grid,
   if (heads == 0 && phi_out == nullptr) return TRA_OK;
   if (heads > 0 && r == nullptr) return TRA_ERR_INVALID_ARGUMENT;
   if (heads > 65535) return TRA_ERR_UNSUPPORTED;
-  const tra_status dv = check_device();
+  const tra_status dv = check_device({r, phi_out});
   if (dv != TRA_OK) return dv;
   // band b = floor(log2(delta + 1)); window factor 2^(-b/2) (disk: the area
   // halves per band) or 2^(-b) (1D: the length halves per band)
@@ -366,9 +375,9 @@ tra_status tra_build_block_mask_ex(const float* r, const float* phi, int heads, 
   if (heads > 65535 || static_cast<long long>(heads) * nqb * nkb >= INT_MAX) return TRA_ERR_UNSUPPORTED;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (heads == 0 || N == 0) {
-    const tra_status dv = check_device();
-    if (dv != TRA_OK) return dv;
     if (heads > 0 && row_ptr == nullptr) return TRA_ERR_INVALID_ARGUMENT;
+    const tra_status dv = check_device({row_ptr, nnz});
+    if (dv != TRA_OK) return dv;
     cudaError_t e = cudaSuccess;
     if (heads > 0) e = cudaMemsetAsync(row_ptr, 0, sizeof(int) * heads, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(nnz, 0, sizeof(int), st);
@@ -380,7 +389,7 @@ tra_status tra_build_block_mask_ex(const float* r, const float* phi, int heads, 
   if (workspace == nullptr || workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return TRA_ERR_WORKSPACE;
-  const tra_status dv = check_device();
+  const tra_status dv = check_device({r, phi, row_ptr, col_idx, nnz, workspace});
   if (dv != TRA_OK) return dv;
   return status_of(launch_block_mask(r, phi, heads, layout_of(grid, tile), block_q, block_k,
                                      vote_threshold, metric == TRA_METRIC_LINE, row_ptr,
@@ -399,7 +408,7 @@ tra_status tra_build_block_mask(const float* r, const float* phi, int heads, tra
 tra_status tra_selftest_wait_timeout(int limit_ms, int* completed, tra_stream_t stream) {
   if (limit_ms < 1 || limit_ms > 2000) return TRA_ERR_INVALID_ARGUMENT;
   if (completed != nullptr && !aligned16(completed)) return TRA_ERR_INVALID_ARGUMENT;
-  const tra_status dv = check_device();
+  const tra_status dv = check_device({completed});
   if (dv != TRA_OK) return dv;
   return status_of(launch_selftest_wait(static_cast<unsigned long long>(limit_ms) * 1000000ull,
                                         completed, reinterpret_cast<cudaStream_t>(stream)));

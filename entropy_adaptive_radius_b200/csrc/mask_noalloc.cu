@@ -21,17 +21,11 @@
 #include <cstdint>
 #include <mutex>
 
-#include <nvtx3/nvToolsExt.h>
 
 #include "tra_internal.h"
 
 namespace tra {
 namespace {
-
-struct NvtxRange {
-  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
-  ~NvtxRange() { nvtxRangePop(); }
-};
 
 constexpr size_t kMaskStaticScratchBytes = static_cast<size_t>(TRA_MASK_STATIC_SCRATCH_BYTES);
 
@@ -74,12 +68,7 @@ extern "C" tra_status tra_build_block_mask_noalloc(const float* r, const float* 
                                                    int* nnz, tra_stream_t stream) {
   using namespace tra;
   NvtxRange nvtx_range("tra_build_block_mask_noalloc");
-  if (heads < 0 || grid.F < 0 || grid.H < 0 || grid.W < 0 || grid.F > kMaxFrames ||
-      grid.H > kMaxSide || grid.W > kMaxSide ||
-      static_cast<long long>(grid.F) * grid.H * grid.W > (1LL << 24) || tile.t < 1 ||
-      tile.y < 1 || tile.x < 1)
-    return TRA_ERR_INVALID_ARGUMENT;
-  auto block_ok = [](int b) { return b == 16 || b == 64 || b == 128; };
+  if (heads < 0 || !grid_ok(grid) || !tile_ok(tile)) return TRA_ERR_INVALID_ARGUMENT;
   if (!block_ok(block_q) || !block_ok(block_k)) return TRA_ERR_UNSUPPORTED;
   if (vote_threshold < 1) return TRA_ERR_INVALID_ARGUMENT;
   if (grid.F > kMaxMaskFrames) return TRA_ERR_UNSUPPORTED;
@@ -89,7 +78,7 @@ extern "C" tra_status tra_build_block_mask_noalloc(const float* r, const float* 
   const long long nqb = (N + block_q - 1) / block_q, nkb = (N + block_k - 1) / block_k;
   if (heads > 65535 || static_cast<long long>(heads) * nqb * nkb >= INT_MAX)
     return TRA_ERR_UNSUPPORTED;
-  const TileLayout L{grid.F, grid.H, grid.W, tile.t, tile.y, tile.x};
+  const TileLayout L = layout_of(grid, tile);
   if (heads > 0 && N > 0) {
     if (r == nullptr || phi == nullptr || row_ptr == nullptr) return TRA_ERR_INVALID_ARGUMENT;
     if (col_idx == nullptr && col_capacity > 0) return TRA_ERR_INVALID_ARGUMENT;
@@ -99,13 +88,8 @@ extern "C" tra_status tra_build_block_mask_noalloc(const float* r, const float* 
   } else if (heads > 0 && row_ptr == nullptr) {
     return TRA_ERR_INVALID_ARGUMENT;
   }
-  int dev = -1, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
-    cudaGetLastError();
-    return TRA_ERR_DEVICE;
-  }
-  if (major != 10) return TRA_ERR_DEVICE;
+  const tra_status dv = check_device({r, phi, row_ptr, col_idx, nnz});
+  if (dv != TRA_OK) return dv;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (heads == 0 || N == 0) {
     cudaError_t e = cudaSuccess;

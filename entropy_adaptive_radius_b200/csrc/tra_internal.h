@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
+#include <initializer_list>
 
 #include "tra.h"
 #include "layout.cuh"
@@ -15,6 +16,22 @@ constexpr int kMaxSide = 16384;    // H, W bound: squared distances stay below 2
 
 // Device error word of the current device (a module-scope __device__ int).
 int* device_error_word();
+
+// Argument checks shared by the entry points (defined in api.cu).
+bool grid_ok(const tra_grid& g);  // sides >= 0, within kMaxFrames / kMaxSide, N <= 2^24
+bool tile_ok(const tra_tile& t);  // every tile side >= 1
+bool block_ok(int b);             // block sizes 16, 64, 128
+TileLayout layout_of(const tra_grid& g, const tra_tile& t);
+// TRA_OK when the current device has compute capability 10.x and every
+// non-null pointer of `ptrs` is device memory of that device (or managed
+// memory); TRA_ERR_DEVICE or TRA_ERR_INVALID_ARGUMENT otherwise.  Host
+// pointers are refused here, before any launch, instead of faulting a kernel.
+tra_status check_device(std::initializer_list<const void*> ptrs = {});
+// NVTX range named after an API call, visible to Nsight tools (no-op without one).
+struct NvtxRange {
+  explicit NvtxRange(const char* name);
+  ~NvtxRange();
+};
 
 // permute.cu
 cudaError_t launch_permute(const void* src, void* dst, tra_dtype in_dtype, tra_dtype out_dtype,

@@ -100,7 +100,13 @@ def _check(fn: str, s: int):
 
 
 def _p(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device pointer of a tensor on the current CUDA device (None stays None)."""
+    if t is None:
+        return None
+    if not t.is_cuda or t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device}: the library takes tensors on the current "
+                         "CUDA device")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream) -> ctypes.c_void_p:

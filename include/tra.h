@@ -16,7 +16,10 @@
  * Conventions shared by every call:
  *  - Pointers are DEVICE pointers owned by the caller unless a comment says
  *    otherwise.  The library never allocates device memory; scratch space is
- *    passed in (see tra_mask_workspace_size).
+ *    passed in (see tra_mask_workspace_size).  Each call asks the CUDA runtime
+ *    where its pointers live and returns TRA_ERR_INVALID_ARGUMENT, launching
+ *    nothing, for host memory (pageable or pinned) or memory of another
+ *    device; managed memory is accepted.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream) and never synchronises, except tra_get_device_error.
  *  - Every call checks its arguments first and launches nothing when it
@@ -44,7 +47,7 @@ typedef struct CUstream_st* tra_stream_t; /* identical to cudaStream_t */
 
 typedef enum {
   TRA_OK = 0,
-  TRA_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misaligned pointer */
+  TRA_ERR_INVALID_ARGUMENT = 1, /* null, misaligned or host pointer, bad size */
   TRA_ERR_UNSUPPORTED = 2,      /* valid but outside the supported shapes */
   TRA_ERR_WORKSPACE = 3,        /* workspace too small or misaligned */
   TRA_ERR_CAPACITY = 4,         /* col_idx capacity negative */

@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 import torch
 
-# spec tolerances: attention output (bf16 inputs, fp32 accumulation),
+# parity tolerances: attention output (bf16 inputs, fp32 accumulation),
 # entropy; LSE follows entropy (both are ln Z up to a bounded term)
 O_MAX_ABS = 2e-2
 O_MEAN_ABS = 2e-3
