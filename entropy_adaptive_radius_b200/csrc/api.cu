@@ -10,6 +10,7 @@
 
 #include <nvtx3/nvToolsExt.h>
 
+#include "ptx.cuh"
 #include "tra_internal.h"
 
 namespace tra {
@@ -111,6 +112,7 @@ const char* tra_status_string(tra_status s) {
     case TRA_ERR_CUDA: return "CUDA runtime error";
     case TRA_ERR_DEVICE: return "no usable compute capability 10.0 (sm_100a) device";
     case TRA_ERR_TIMEOUT: return "a device-side wait ran out of time";
+    case TRA_ERR_BAD_INPUT: return "a kernel met an invalid CSR row (skipped)";
   }
   return "unknown status";
 }
@@ -430,7 +432,8 @@ tra_status tra_get_device_error(int* code, tra_stream_t stream) {
     if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return TRA_ERR_CUDA;
   }
   *code = v;
-  return v != 0 ? TRA_ERR_TIMEOUT : TRA_OK;
+  if (v == 0) return TRA_OK;
+  return v == kErrBadCsr ? TRA_ERR_BAD_INPUT : TRA_ERR_TIMEOUT;
 }
 
 }  // extern "C"

@@ -24,7 +24,7 @@ METRICS = {"disk": TRA_METRIC_DISK, "line": TRA_METRIC_LINE}
 BUDGETS = {"entropy": TRA_BUDGET_ENTROPY, "shared": TRA_BUDGET_SHARED}
 STATUS = {0: "TRA_OK", 1: "TRA_ERR_INVALID_ARGUMENT", 2: "TRA_ERR_UNSUPPORTED",
           3: "TRA_ERR_WORKSPACE", 4: "TRA_ERR_CAPACITY", 5: "TRA_ERR_CUDA",
-          6: "TRA_ERR_DEVICE", 7: "TRA_ERR_TIMEOUT"}
+          6: "TRA_ERR_DEVICE", 7: "TRA_ERR_TIMEOUT", 8: "TRA_ERR_BAD_INPUT"}
 
 
 class TraError(RuntimeError):
@@ -305,7 +305,7 @@ def tra_get_device_error(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device error code."""
     code = _c_int(0)
     s = lib().tra_get_device_error(ctypes.byref(code), _stream(stream))
-    if s not in (0, 7):
+    if s not in (0, 7, 8):
         _check("tra_get_device_error", s)
     return code.value
 

@@ -30,7 +30,9 @@
  *  - Calls on distinct streams may run concurrently from several threads.
  *  - A device-side wait that runs out of time (it never should) makes the
  *    kernel record a code in a device error word and return early; the next
- *    tra_get_device_error reports it.  No kernel traps.
+ *    tra_get_device_error reports it.  A CSR row that a kernel finds invalid
+ *    is skipped (its queries get O = 0, lse = -inf) and recorded the same
+ *    way.  No kernel traps.
  *  - Requires a compute capability 10.0 GPU (B200, sm_100a).
  */
 #ifndef TRA_H_
@@ -53,7 +55,9 @@ typedef enum {
   TRA_ERR_CAPACITY = 4,         /* col_idx capacity negative */
   TRA_ERR_CUDA = 5,             /* a CUDA runtime call failed (launch, attribute) */
   TRA_ERR_DEVICE = 6,           /* no usable sm_100 device */
-  TRA_ERR_TIMEOUT = 7           /* reported by tra_get_device_error */
+  TRA_ERR_TIMEOUT = 7,          /* reported by tra_get_device_error: a wait ran out of time */
+  TRA_ERR_BAD_INPUT = 8         /* reported by tra_get_device_error: a kernel met an invalid
+                                   CSR row (negative start, or longer than nKB) */
 } tra_status;
 
 typedef enum { TRA_BF16 = 0, TRA_F32 = 1 } tra_dtype;
@@ -363,8 +367,15 @@ tra_status tra_selftest_wait_timeout(int limit_ms, int* completed, tra_stream_t 
 /*
  * Synchronises `stream`, then reads and clears the device error word of the
  * current device.  *code = 0 when no kernel recorded an error; otherwise the
- * code of the first wait that ran out of time.  Returns TRA_ERR_TIMEOUT when
- * *code != 0, TRA_ERR_CUDA when the stream reported a CUDA error.
+ * first code recorded:
+ *    1 .. 9  a wait that ran out of time (1 Q tile, 2 / 3 K / V tile loaded,
+ *            4 / 5 K / V stage free, 6 scores ready, 7 score buffer free,
+ *            8 probabilities ready, 9 PV product done)  -> TRA_ERR_TIMEOUT
+ *    10      an invalid CSR row (negative start, or longer than nKB; the
+ *            row is skipped)                              -> TRA_ERR_BAD_INPUT
+ *    11      the self-test's wait (tra_selftest_wait_timeout) -> TRA_ERR_TIMEOUT
+ * Returns TRA_OK when *code == 0, TRA_ERR_CUDA when the stream reported a
+ * CUDA error.
  */
 tra_status tra_get_device_error(int* code, tra_stream_t stream);
 

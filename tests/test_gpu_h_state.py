@@ -70,3 +70,61 @@ def test_layer_state_round_trip_resumes_bit_for_bit():
     c = TraLayer(grid, heads, d, tau=0.3, gamma=0.3, block_q=64, block_k=64, policy=policy)
     with pytest.raises(ValueError):
         c.load_state_dict(a.state_dict())
+
+
+def bad_csr_case(N, B, bad_row, kind):
+    """A CSR over nqb x nkb blocks whose row `bad_row` is invalid (longer
+    than nkb, or with a negative start) and every other row keeps one key
+    block.  Returns (row_ptr, col_idx, mask of what a valid call computes)."""
+    nb = -(-N // B)
+    rows = [[(q + 1) % nb] for q in range(nb)]
+    rp, ci = [0], []
+    for q in range(nb):
+        if q == bad_row and kind == "long":
+            ci += list(range(nb)) + [0]              # nkb + 1 entries
+        else:
+            ci += rows[q]
+        rp.append(len(ci))
+    rp = np.array(rp, np.int32)
+    if kind == "negative":
+        rp[bad_row] = -3                             # start of the bad row
+    mask = np.zeros((1, nb, nb), bool)
+    for q in range(nb):
+        if q != bad_row:
+            mask[0, q, rows[q][0]] = True
+    return rp, np.array(ci, np.int32), mask
+
+
+@pytest.mark.parametrize("B", [128, 64, 16])
+@pytest.mark.parametrize("kind", ["long", "negative"])
+def test_invalid_csr_row_is_skipped_and_reported(B, kind):
+    need_gpu()
+    N, d = 256, 64
+    g = torch.Generator().manual_seed(B)
+    Q, K, V = (torch.randn(1, N, d, generator=g).to(torch.bfloat16) for _ in range(3))
+    # a negative start of row q also ends row q - 1 below its start, so the
+    # negative case uses row 0; the long case a middle row
+    bad = 0 if kind == "negative" else 1
+    rp, ci, mask = bad_csr_case(N, B, bad, kind)
+    O_ = torch.full((1, N, d), 7.0, dtype=torch.bfloat16, device="cuda")
+    L = torch.empty(1, N, device="cuda")
+    assert tra.tra_get_device_error() == 0
+    tra.tra_block_sparse_attn(Q.cuda(), K.cuda(), V.cuda(), O_, torch.from_numpy(rp).cuda(),
+                              torch.from_numpy(ci).cuda(), B, B, lse=L)
+    code = _c_code()
+    assert code == (10, 8)                           # invalid CSR row, TRA_ERR_BAD_INPUT
+    Or, Lr = O.sparse_attention(to64(Q), to64(K), to64(V), mask, B, B, 1.0 / math.sqrt(d))
+    rows = slice(bad * B, (bad + 1) * B)
+    assert bool((O_[0, rows] == 0).all())
+    assert bool(torch.isneginf(L[0, rows]).all())
+    check_attention(O_, Or, f"O with an invalid row ({kind}, B={B})")
+    keep = np.isfinite(Lr[0])
+    assert np.allclose(to64(L)[0, keep], Lr[0, keep], atol=1e-3, rtol=0)
+
+
+def _c_code():
+    """(device code, status) read through the C call itself."""
+    import ctypes
+    code = ctypes.c_int(0)
+    s = tra.lib().tra_get_device_error(ctypes.byref(code), tra._stream(None))
+    return code.value, s
