@@ -137,10 +137,45 @@ def _contig(*ts):
             raise ValueError("tensors must be contiguous")
 
 
+def _want(name: str, t: Optional[torch.Tensor], shape=None, dtypes=None, min_numel=None):
+    """The C calls cannot see allocation sizes, so every tensor's shape and
+    dtype is checked here against the call's dimensions before its pointer
+    is passed on (a short tensor would send a kernel past its end)."""
+    if t is None:
+        return
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name}: {t.numel()} elements, at least {min_numel} needed")
+
+
+_BF16 = (torch.bfloat16,)
+_F32 = (torch.float32,)
+_I32 = (torch.int32,)
+_U8 = (torch.uint8,)
+
+
+def _n_of(grid: Sequence[int]) -> int:
+    F, H, W = (int(v) for v in grid)
+    return F * H * W
+
+
+def _qkv(Q) -> tuple:
+    if Q.dim() != 3:
+        raise ValueError(f"expected [heads, N, d], got shape {tuple(Q.shape)}")
+    return tuple(Q.shape)
+
+
 def tra_tile_major_permute(X, X_tm, grid, tile=(1, 4, 4), stream=None):
     """X_tm[h, p] = X[h, pi(p)] for X [heads, N, d] (bf16 or f32)."""
     _contig(X, X_tm)
-    heads, _, d = X.shape
+    heads, N, d = _qkv(X)
+    if N != _n_of(grid):
+        raise ValueError(f"X has {N} tokens, the grid {tuple(grid)} has {_n_of(grid)}")
+    _want("X", X, dtypes=_BF16 + _F32)
+    _want("X_tm", X_tm, (heads, N, d), _BF16 + _F32)
     _check("tra_tile_major_permute", lib().tra_tile_major_permute(
         _p(X), _p(X_tm), _dtype(X), _dtype(X_tm), heads, d, _grid(grid), _tile(tile),
         _stream(stream)))
@@ -152,7 +187,11 @@ def tra_inverse_permute(X_tm, X, grid, tile=(1, 4, 4), stream=None):
     _contig(X, X_tm)
     if X.dtype != X_tm.dtype:
         raise TypeError("inverse permute keeps the dtype")
-    heads, _, d = X_tm.shape
+    heads, N, d = _qkv(X_tm)
+    if N != _n_of(grid):
+        raise ValueError(f"X_tm has {N} tokens, the grid {tuple(grid)} has {_n_of(grid)}")
+    _want("X_tm", X_tm, dtypes=_BF16 + _F32)
+    _want("X", X, (heads, N, d))
     _check("tra_inverse_permute", lib().tra_inverse_permute(
         _p(X_tm), _p(X), _dtype(X_tm), heads, d, _grid(grid), _tile(tile), _stream(stream)))
     return X
@@ -161,7 +200,11 @@ def tra_inverse_permute(X_tm, X, grid, tile=(1, 4, 4), stream=None):
 def tra_dense_attn_entropy(Q, K, V, O, H, lse=None, scale=None, stream=None):
     """Dense attention O, entropy H and (optionally) LSE of Q, K, V [heads, N, d] bf16."""
     _contig(Q, K, V, O, H, lse)
-    heads, N, d = Q.shape
+    heads, N, d = _qkv(Q)
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("O", O)):
+        _want(name, t, (heads, N, d), _BF16)
+    _want("H", H, (heads, N), _F32)
+    _want("lse", lse, (heads, N), _F32)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     _check("tra_dense_attn_entropy", lib().tra_dense_attn_entropy(
         _p(Q), _p(K), _p(V), _p(O), _p(H), _p(lse), heads, N, d, scale, _stream(stream)))
@@ -172,17 +215,29 @@ def tra_attn_entropy(Q, K, H, lse=None, scale=None, stream=None):
     """Entropy H (and optionally LSE) of every query of Q, K [heads, N, d] bf16
     over all keys, without the PV product or an output."""
     _contig(Q, K, H, lse)
-    heads, N, d = Q.shape
+    heads, N, d = _qkv(Q)
+    _want("Q", Q, (heads, N, d), _BF16)
+    _want("K", K, (heads, N, d), _BF16)
+    _want("H", H, (heads, N), _F32)
+    _want("lse", lse, (heads, N), _F32)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     _check("tra_attn_entropy", lib().tra_attn_entropy(
         _p(Q), _p(K), _p(H), _p(lse), heads, N, d, scale, _stream(stream)))
     return H
 
 
+def _radius_args(heads, grid, H, r, phi_out):
+    N = _n_of(grid)
+    _want("H", H, (heads, N), _F32)
+    _want("r", r, (heads, N), _F32)
+    _want("phi_out", phi_out, dtypes=_F32, min_numel=int(grid[0]))
+
+
 def tra_budget_radius(H, r, grid, tau, gamma, tile=(1, 4, 4), phi_out=None, stream=None):
     """Per-query base radius r [heads, N] from entropy H (tile-major order)."""
     _contig(H, r, phi_out)
     heads = H.shape[0]
+    _radius_args(heads, grid, H, r, phi_out)
     _check("tra_budget_radius", lib().tra_budget_radius(
         _p(H), _p(r), _p(phi_out), heads, _grid(grid), _tile(tile), float(tau), float(gamma),
         _stream(stream)))
@@ -195,6 +250,7 @@ def tra_budget_radius_ex(H, r, grid, tau, gamma, budget="entropy", metric="disk"
     "shared" per head) and distance ("disk", "line")."""
     _contig(H, r, phi_out)
     heads = H.shape[0]
+    _radius_args(heads, grid, H, r, phi_out)
     _check("tra_budget_radius_ex", lib().tra_budget_radius_ex(
         _p(H), _p(r), _p(phi_out), heads, _grid(grid), _tile(tile), float(tau), float(gamma),
         BUDGETS[budget], METRICS[metric], _stream(stream)))
@@ -205,10 +261,22 @@ def tra_radial_radius(r, grid, r0, metric="disk", tile=(1, 4, 4), phi_out=None, 
     """Radial Attention's static window: r = r0 everywhere and the band table in phi_out."""
     _contig(r, phi_out)
     heads = r.shape[0]
+    _radius_args(heads, grid, None, r, phi_out)
     _check("tra_radial_radius", lib().tra_radial_radius(
         _p(r), _p(phi_out), heads, _grid(grid), _tile(tile), float(r0), METRICS[metric],
         _stream(stream)))
     return r
+
+
+def _mask_args(heads, grid, block_q, block_k, r, phi, row_ptr, col_idx, nnz, workspace=None):
+    N = _n_of(grid)
+    nqb = -(-N // block_q) if block_q > 0 else 0
+    _want("r", r, (heads, N), _F32)
+    _want("phi", phi, dtypes=_F32, min_numel=int(grid[0]))
+    _want("row_ptr", row_ptr, dtypes=_I32, min_numel=heads * (nqb + 1))
+    _want("col_idx", col_idx, dtypes=_I32)
+    _want("nnz", nnz, dtypes=_I32, min_numel=1)
+    _want("workspace", workspace, dtypes=_U8)
 
 
 def tra_mask_workspace_size(heads, grid, block_q, block_k, tile=(1, 4, 4)) -> int:
@@ -221,6 +289,7 @@ def tra_build_block_mask(r, phi, grid, block_q, block_k, vote, row_ptr, col_idx,
     at least tra_mask_workspace_size bytes (256-byte aligned)."""
     _contig(r, phi, row_ptr, col_idx, nnz, workspace)
     heads = r.shape[0]
+    _mask_args(heads, grid, block_q, block_k, r, phi, row_ptr, col_idx, nnz, workspace)
     _check("tra_build_block_mask", lib().tra_build_block_mask(
         _p(r), _p(phi), heads, _grid(grid), _tile(tile), block_q, block_k, vote, _p(row_ptr),
         _p(col_idx), col_idx.numel(), _p(nnz), _p(workspace), workspace.numel(),
@@ -233,6 +302,7 @@ def tra_build_block_mask_ex(r, phi, grid, block_q, block_k, vote, row_ptr, col_i
     """tra_build_block_mask with a choice of distance ("disk" or "line")."""
     _contig(r, phi, row_ptr, col_idx, nnz, workspace)
     heads = r.shape[0]
+    _mask_args(heads, grid, block_q, block_k, r, phi, row_ptr, col_idx, nnz, workspace)
     _check("tra_build_block_mask_ex", lib().tra_build_block_mask_ex(
         _p(r), _p(phi), heads, _grid(grid), _tile(tile), block_q, block_k, vote, METRICS[metric],
         _p(row_ptr), _p(col_idx), col_idx.numel(), _p(nnz), _p(workspace), workspace.numel(),
@@ -248,6 +318,7 @@ def tra_build_block_mask_noalloc(r, phi, grid, block_q, block_k, vote, row_ptr, 
     race; issue them in order on one stream."""
     _contig(r, phi, row_ptr, col_idx, nnz)
     heads = r.shape[0]
+    _mask_args(heads, grid, block_q, block_k, r, phi, row_ptr, col_idx, nnz)
     _check("tra_build_block_mask_noalloc", lib().tra_build_block_mask_noalloc(
         _p(r), _p(phi), heads, _grid(grid), _tile(tile), block_q, block_k, vote, _p(row_ptr),
         _p(col_idx), col_idx.numel(), _p(nnz), _stream(stream)))
@@ -257,11 +328,21 @@ def tra_build_block_mask_noalloc(r, phi, grid, block_q, block_k, vote, row_ptr, 
 MASK_STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 
+def _csr_args(heads, N, block_q, row_ptr, col_idx, lse):
+    nqb = -(-N // block_q) if block_q > 0 else 0
+    _want("row_ptr", row_ptr, dtypes=_I32, min_numel=heads * (nqb + 1))
+    _want("col_idx", col_idx, dtypes=_I32)
+    _want("lse", lse, (heads, N), _F32)
+
+
 def tra_block_sparse_attn(Q, K, V, O, row_ptr, col_idx, block_q, block_k, lse=None, scale=None,
                           stream=None):
     """Exact attention over the kept blocks of the CSR mask."""
     _contig(Q, K, V, O, row_ptr, col_idx, lse)
-    heads, N, d = Q.shape
+    heads, N, d = _qkv(Q)
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("O", O)):
+        _want(name, t, (heads, N, d), _BF16)
+    _csr_args(heads, N, block_q, row_ptr, col_idx, lse)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     _check("tra_block_sparse_attn", lib().tra_block_sparse_attn(
         _p(Q), _p(K), _p(V), _p(O), _p(lse), _p(row_ptr), _p(col_idx), heads, N, d, block_q,
@@ -273,9 +354,10 @@ def tra_quantize_e4m3(X, Xq, scales, block=128, stream=None):
     """Per-block E4M3 codes Xq (uint8 [heads, N, d]) and fp32 scales
     [heads, ceil(N / block)] of a bf16 X [heads, N, d]."""
     _contig(X, Xq, scales)
-    heads, N, d = X.shape
-    if Xq.dtype != torch.uint8:
-        raise TypeError("Xq holds E4M3 codes as uint8")
+    heads, N, d = _qkv(X)
+    _want("X", X, (heads, N, d), _BF16)
+    _want("Xq", Xq, (heads, N, d), _U8)
+    _want("scales", scales, (heads, -(-N // block) if block > 0 else 0), _F32)
     _check("tra_quantize_e4m3", lib().tra_quantize_e4m3(
         _p(X), _p(Xq), _p(scales), heads, N, d, block, _stream(stream)))
     return Xq, scales
@@ -285,7 +367,15 @@ def tra_block_sparse_attn_fp8(Q8, q_scales, K8, k_scales, V, O, row_ptr, col_idx
                               block_k=128, lse=None, scale=None, stream=None):
     """Block-sparse attention with E4M3 Q and K (from tra_quantize_e4m3, block 128)."""
     _contig(Q8, q_scales, K8, k_scales, V, O, row_ptr, col_idx, lse)
-    heads, N, d = V.shape
+    heads, N, d = _qkv(V)
+    _want("Q8", Q8, (heads, N, d), _U8)
+    _want("K8", K8, (heads, N, d), _U8)
+    _want("V", V, (heads, N, d), _BF16)
+    _want("O", O, (heads, N, d), _BF16)
+    nsc = -(-N // 128)
+    _want("q_scales", q_scales, (heads, nsc), _F32)
+    _want("k_scales", k_scales, (heads, nsc), _F32)
+    _csr_args(heads, N, block_q, row_ptr, col_idx, lse)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     _check("tra_block_sparse_attn_fp8", lib().tra_block_sparse_attn_fp8(
         _p(Q8), _p(q_scales), _p(K8), _p(k_scales), _p(V), _p(O), _p(lse), _p(row_ptr),
@@ -297,6 +387,7 @@ def tra_selftest_wait_timeout(limit_ms, completed=None, stream=None):
     """Launch the bounded-wait self-test (a wait that nothing completes, given
     up after limit_ms); read the outcome with tra_get_device_error."""
     _contig(completed)
+    _want("completed", completed, dtypes=_I32, min_numel=1)
     _check("tra_selftest_wait_timeout", lib().tra_selftest_wait_timeout(
         int(limit_ms), _p(completed), _stream(stream)))
 
