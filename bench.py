@@ -883,6 +883,8 @@ def kernel_case(args):
     dense / sparse / entropy (entropy only, no PV) / sparse_fp8 (E4M3 Q, K) /
     quant (E4M3 quantization of Q): 40 heads x 16384 tokens x d=128 bf16
     (168 MB per tensor);
+    sparse64: the Wan2.1-1.3B shape (12 x 32760 x 128, 64-token blocks) on its
+    own radius mask at the calibrated kept fraction;
     mask: the 21x45x80 grid, 40 heads, radii from entropies near ln N;
     permute: one 21x45x80 x 40-head x 128 bf16 tensor.  Runs the kernel
     `--reps` times and prints the mean CUDA-event time per launch."""
@@ -892,7 +894,23 @@ def kernel_case(args):
     g = torch.Generator(device=dev).manual_seed(0)
     heads, N, d = 40, 16384, 128
     reps = args.reps
-    if args.case in ("dense", "sparse", "sparse_fp8", "quant", "entropy"):
+    if args.case == "sparse64":
+        # the Wan2.1-1.3B shape with its own radius mask (64-token blocks, so
+        # each 128-row tile runs the union of two query blocks' rows)
+        wl = workloads.WAN13B
+        Q, K, V = (t.to(dev) for t in inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed,
+                                                      wl.q_scale, "bf16"))
+        pipe = Pipeline(wl, dev)
+        pipe.warmup_call(Q, K, V, None)
+        pipe.mask(calibrate_tau(pipe, wl.kept_target, lambda m: print(f"[bench] {m}", file=sys.stderr)))
+        rp_h = pipe.row_ptr.cpu().numpy()
+        ci_h = pipe.col_idx.cpu().numpy()
+        flops = 4.0 * wl.d * kept_pair_tokens(rp_h, ci_h, wl.heads, wl.N, wl.block_q, wl.block_k)
+        q, k, v, o = pipe.Qtm, pipe.Ktm, pipe.Vtm, pipe.Otm
+        fn = lambda: tra.tra_block_sparse_attn(q, k, v, o, pipe.row_ptr, pipe.col_idx,  # noqa: E731
+                                               wl.block_q, wl.block_k)
+        unit = ("TFLOP/s", flops / 1e12)
+    elif args.case in ("dense", "sparse", "sparse_fp8", "quant", "entropy"):
         Q = (torch.randn(heads, N, d, generator=g, device=dev) * 2).to(torch.bfloat16)
         K = torch.randn(heads, N, d, generator=g, device=dev).to(torch.bfloat16)
         V = torch.randn(heads, N, d, generator=g, device=dev).to(torch.bfloat16)
@@ -965,7 +983,7 @@ def kernel_case(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["dense", "sparse", "sparse_fp8", "quant", "entropy", "mask",
+    ap.add_argument("--case", choices=["dense", "sparse", "sparse64", "sparse_fp8", "quant", "entropy", "mask",
                                        "permute"], default=None,
                     help="run one kernel on a small case (for profiler captures)")
     ap.add_argument("--reps", type=int, default=3)

@@ -775,15 +775,10 @@ __global__ void __launch_bounds__(kDualThreads, 1)
           if (p.err) atomicCAS(p.err, 0, kErrBadCsr);
         }
       }
-      int total = n[0];
-      if (n[1] > 0) {
-        ListWalker wk{p.col_idx + st[0], p.col_idx + st[1], n[0], n[1], 0, 0};
-        uint32_t mem;
-        total = 0;
-        while (wk.next(mem) >= 0) ++total;
-      }
-      misc[2] = (total + E - 1) / E;
+      // two query blocks: the union's length is set below, by all threads
+      misc[2] = (n[0] + E - 1) / E;
       misc[3] = st[0]; misc[4] = n[0]; misc[5] = st[1]; misc[6] = n[1];
+      misc[7] = 0;
     }
   }
   if (warp == kDualKWarp) {
@@ -796,6 +791,37 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     }
   }
   __syncthreads();
+  if constexpr (!DENSE) {
+    if (misc[6] > 0) {
+      // Length of the merged list of two ascending CSR rows A and B:
+      // |A| + |B| - |A and B|, counted in parallel with a bitmap of A's key
+      // blocks in P_0 (free until the first probabilities are stored; it
+      // holds 262144 bits, the largest nKB).
+      static_assert(C::P_BYTES * 8 >= (1 << 24) / 64, "key-block bitmap");
+      const int na = misc[4], nb = misc[6];
+      const int* a = p.col_idx + misc[3];
+      const int* b = p.col_idx + misc[5];
+      uint32_t* bm = reinterpret_cast<uint32_t*>(smem + C::OFF_P);
+      const int nw = (p.nkb + 31) >> 5;
+      for (int i = tid; i < nw; i += kDualThreads) bm[i] = 0u;
+      __syncthreads();
+      for (int i = tid; i < na; i += kDualThreads) {
+        const int kb = __ldg(a + i);
+        if (kb >= 0 && kb < p.nkb) atomicOr(bm + (kb >> 5), 1u << (kb & 31));
+      }
+      __syncthreads();
+      int both = 0;
+      for (int i = tid; i < nb; i += kDualThreads) {
+        const int kb = __ldg(b + i);
+        if (kb >= 0 && kb < p.nkb) both += static_cast<int>((bm[kb >> 5] >> (kb & 31)) & 1u);
+      }
+      both = __reduce_add_sync(0xffffffffu, both);
+      if (lane == 0 && both > 0) atomicAdd(const_cast<int*>(misc + 7), both);
+      __syncthreads();
+      if (tid == 0) misc[2] = (na + nb - misc[7] + E - 1) / E;
+      __syncthreads();
+    }
+  }
   tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
   const int nblk = misc[2];  // super-blocks
