@@ -657,7 +657,11 @@ struct DualCfg {
   static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
   static constexpr int NUM_BARS = 1 + 4 * NS + 8 + 2;
   static constexpr int OFF_MISC = OFF_BAR + 256;
-  static constexpr int USED = OFF_MISC + 64;
+  // merged key-block list of a tile's two query blocks (entries with their
+  // membership bits), when it has at most kUnionCap entries
+  static constexpr int kUnionCap = 384;
+  static constexpr int OFF_LIST = OFF_MISC + 64;
+  static constexpr int USED = OFF_LIST + kUnionCap * 4;
   static constexpr int SMEM = (USED < 120 * 1024 ? 120 * 1024 : USED) + 1024;
   static constexpr int TMEM_COLS = 512;  // S_0, S_1 (128 each), O_0, O_1 (D each)
   static_assert(2 * BK + 2 * D <= TMEM_COLS, "tensor memory");
@@ -779,6 +783,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       misc[2] = (n[0] + E - 1) / E;
       misc[3] = st[0]; misc[4] = n[0]; misc[5] = st[1]; misc[6] = n[1];
       misc[7] = 0;
+      misc[8] = 0;  // 1: the merged list is in shared memory
     }
   }
   if (warp == kDualKWarp) {
@@ -793,32 +798,72 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   __syncthreads();
   if constexpr (!DENSE) {
     if (misc[6] > 0) {
-      // Length of the merged list of two ascending CSR rows A and B:
-      // |A| + |B| - |A and B|, counted in parallel with a bitmap of A's key
-      // blocks in P_0 (free until the first probabilities are stored; it
-      // holds 262144 bits, the largest nKB).
+      // Merged list of two ascending CSR rows A and B.  Its length is
+      // |A| + |B| - |A and B|, counted in parallel from bitmaps of A's and B's
+      // key blocks in P_0 and P_1 (free until the first probabilities are
+      // stored; each holds 262144 bits, the largest nKB).  A list of at most
+      // kUnionCap entries is then written out in order, with membership bits,
+      // so the softmax reads its entries instead of walking the two rows.
       static_assert(C::P_BYTES * 8 >= (1 << 24) / 64, "key-block bitmap");
       const int na = misc[4], nb = misc[6];
       const int* a = p.col_idx + misc[3];
       const int* b = p.col_idx + misc[5];
-      uint32_t* bm = reinterpret_cast<uint32_t*>(smem + C::OFF_P);
+      uint32_t* bma = reinterpret_cast<uint32_t*>(smem + C::OFF_P);
+      uint32_t* bmb = reinterpret_cast<uint32_t*>(smem + C::OFF_P + C::P_BYTES);
       const int nw = (p.nkb + 31) >> 5;
-      for (int i = tid; i < nw; i += kDualThreads) bm[i] = 0u;
+      for (int i = tid; i < nw; i += kDualThreads) {
+        bma[i] = 0u;
+        bmb[i] = 0u;
+      }
       __syncthreads();
       for (int i = tid; i < na; i += kDualThreads) {
         const int kb = __ldg(a + i);
-        if (kb >= 0 && kb < p.nkb) atomicOr(bm + (kb >> 5), 1u << (kb & 31));
+        if (kb >= 0 && kb < p.nkb) atomicOr(bma + (kb >> 5), 1u << (kb & 31));
       }
       __syncthreads();
       int both = 0;
       for (int i = tid; i < nb; i += kDualThreads) {
         const int kb = __ldg(b + i);
-        if (kb >= 0 && kb < p.nkb) both += static_cast<int>((bm[kb >> 5] >> (kb & 31)) & 1u);
+        if (kb >= 0 && kb < p.nkb) {
+          both += static_cast<int>((bma[kb >> 5] >> (kb & 31)) & 1u);
+          atomicOr(bmb + (kb >> 5), 1u << (kb & 31));
+        }
       }
       both = __reduce_add_sync(0xffffffffu, both);
       if (lane == 0 && both > 0) atomicAdd(const_cast<int*>(misc + 7), both);
       __syncthreads();
-      if (tid == 0) misc[2] = (na + nb - misc[7] + E - 1) / E;
+      const int ulen = na + nb - misc[7];
+      if (tid == 0) {
+        misc[2] = (ulen + E - 1) / E;
+        misc[9] = ulen;
+      }
+      if (ulen <= C::kUnionCap && warp == 0) {
+        // warp 0 writes the set bits of A | B in ascending order, 32 words a round
+        uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
+        int run = 0;
+        for (int base = 0; base < nw; base += 32) {
+          const int wd = base + lane;
+          const uint32_t wa = wd < nw ? bma[wd] : 0u, wb = wd < nw ? bmb[wd] : 0u;
+          uint32_t word = wa | wb;
+          const int cnt = __popc(word);
+          int incl = cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+          }
+          int pos = run + incl - cnt;
+          while (word) {
+            const int bit = __ffs(word) - 1;
+            word &= word - 1;
+            const uint32_t mem = ((wa >> bit) & 1u) | (((wb >> bit) & 1u) << 1);
+            if (pos < C::kUnionCap) list[pos] = static_cast<uint32_t>(wd * 32 + bit) | (mem << 30);
+            ++pos;
+          }
+          run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) misc[8] = 1;
+      }
       __syncthreads();
     }
   }
@@ -994,6 +1039,14 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     // entry, so entry j is simply the j-th list element (one load, no walk)
     constexpr bool kDirect = (E == 1) && (DENSE || SINGLE);
     const int* my_list = p.col_idx + misc[3];
+    // Otherwise entry j * E + e comes from: the tile's one CSR row (read
+    // directly, entries of query block A), or the merged list in shared
+    // memory, or, when that list would not fit, a walk of the two rows.
+    const bool one_row = SINGLE || misc[6] == 0;
+    const int n_row = misc[4];
+    const bool use_list = !one_row && misc[8] != 0;
+    const int ulen = misc[9];
+    const uint32_t* s_list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
     // FP8 scores carry the query block's and the key block's scale
     float q_sl2 = p.scale_log2;
     if constexpr (FP8) q_sl2 *= __ldg(p.q_scales + static_cast<size_t>(h) * p.nqb + qt);
@@ -1008,6 +1061,23 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         nv[0] = kb_ok ? min(BKS, p.N - kb * BKS) : 0;
         if constexpr (FP8) {
           if (kb_ok) sl2 *= __ldg(p.k_scales + static_cast<size_t>(h) * p.nkb + kb);
+        }
+      } else if (one_row) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int idx = j * E + e;
+          const int kb = idx < n_row ? __ldg(my_list + idx) : -1;
+          const bool keep = kb >= 0 && kb < p.nkb && (my_bit & 1u) != 0u;
+          nv[e] = keep ? min(BKS, p.N - kb * BKS) : 0;
+        }
+      } else if (use_list) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int idx = j * E + e;
+          const uint32_t ent = idx < ulen ? s_list[idx] : 0xFFFFFFFFu;
+          const int kb = ent == 0xFFFFFFFFu ? -1 : static_cast<int>(ent & 0x3FFFFFFFu);
+          const bool keep = kb >= 0 && kb < p.nkb && ((ent >> 30) & my_bit) != 0u;
+          nv[e] = keep ? min(BKS, p.N - kb * BKS) : 0;
         }
       } else {
         // walk the merged list, skipping the other warpgroup's super-blocks
@@ -1097,7 +1167,22 @@ __global__ void __launch_bounds__(kDualThreads, 1)
 #pragma unroll
         for (int c8 = 0; c8 < BK / 8; ++c8) st_shared_v4(prow + poff[c8], 0u, 0u, 0u, 0u);
       } else {
-        if (mode == 2) {
+        // Two 64-key entries: each half of the super-block is kept whole or
+        // not at all by this warp's query block, except in the sequence's last
+        // key block.  Whole halves need no per-key mask: an unkept half is left
+        // out of the max and gets offset -inf below (x = -inf, p = 0).
+        bool halves = false;
+        bool keep_half[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) keep_half[e] = true;
+        if constexpr (E == 2) {
+          halves = (nv[0] == 0 || nv[0] == BKS) && (nv[1] == 0 || nv[1] == BKS);
+          if (halves) {
+            keep_half[0] = nv[0] > 0;
+            keep_half[1] = nv[1] > 0;
+          }
+        }
+        if (mode == 2 && !halves) {
           // partly valid: invalid keys (past N, or not kept by this row's
           // query block) get a huge negative score, so p = 0 and p * x = 0
           // without special cases; a row with no valid key leaves its
@@ -1107,30 +1192,54 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         }
         {
           // row max: 16 independent chains of 3-input max, then a small tree
-          float mx[16];
+          // (per 64-key half with two entries)
+          float bmax;
+          if constexpr (E == 2) {
+            float hm[2];
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            mx[q] = fmax3(sv[q], sv[16 + q], sv[32 + q]);
-            mx[q] = fmax3(mx[q], sv[48 + q], sv[64 + q]);
-            mx[q] = fmax3(mx[q], sv[80 + q], sv[96 + q]);
-            mx[q] = fmaxf(mx[q], sv[112 + q]);
+            for (int e = 0; e < 2; ++e) {
+              float mx[16];
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                mx[q] = fmax3(sv[64 * e + q], sv[64 * e + 16 + q], sv[64 * e + 32 + q]);
+                mx[q] = fmaxf(mx[q], sv[64 * e + 48 + q]);
+              }
+#pragma unroll
+              for (int q = 0; q < 5; ++q) mx[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
+              hm[e] = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[15]));
+              if (!keep_half[e]) hm[e] = -INFINITY;
+            }
+            bmax = fmaxf(hm[0], hm[1]);
+          } else {
+            float mx[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              mx[q] = fmax3(sv[q], sv[16 + q], sv[32 + q]);
+              mx[q] = fmax3(mx[q], sv[48 + q], sv[64 + q]);
+              mx[q] = fmax3(mx[q], sv[80 + q], sv[96 + q]);
+              mx[q] = fmaxf(mx[q], sv[112 + q]);
+            }
+#pragma unroll
+            for (int q = 0; q < 5; ++q) mx[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
+            bmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[15]));
           }
-#pragma unroll
-          for (int q = 0; q < 5; ++q) mx[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
-          const float m6 = fmax3(mx[0], mx[1], mx[2]);
-          const float m7 = fmax3(mx[3], mx[4], mx[15]);
-          if (any_valid) update_max(fmaxf(m6, m7) * sl2);
+          if (any_valid) update_max(bmax * sl2);
         }
         // x = s * scale * log2(e) - m_ref, p = 2^x, Z += p, A += p * x, two
         // lanes per instruction (m_ref is -inf only for a row with no valid
-        // key yet, whose p are then all 0)
+        // key yet, whose p are then all 0); an unkept half's offset is -inf
         const float2 sc2 = make_float2(sl2, sl2);
         const float mc = (m_ref == -INFINITY) ? 0.f : m_ref;
-        const float2 nm2 = make_float2(-mc, -mc);
+        float2 nmh[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const float o = keep_half[e] ? -mc : -INFINITY;
+          nmh[e] = make_float2(o, o);
+        }
         float2 z2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         auto pair = [&](int c) -> uint32_t {
-          const float2 x = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nm2);
+          const float2 x = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nmh[(2 * c) / BKS]);
           const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           z2[c & 1] = __fadd2_rn(z2[c & 1], pr);
           if constexpr (DENSE) a2[c & 1] = __ffma2_rn(pr, x, a2[c & 1]);
