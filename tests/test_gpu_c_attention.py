@@ -210,3 +210,35 @@ def test_full_size_dense_and_sparse_sampled(wl):
     assert bool(torch.isfinite(O_).all()) and bool(torch.isfinite(Os).all())
     assert np.isfinite(Hn).all()
     assert (Hn <= math.log(N) + H_ABS).all() and (Hn >= -H_ABS).all()
+
+
+def test_union_list_and_walk_fallback_at_the_cap():
+    """64-row query blocks pair up in 128-row tiles whose key-block list is
+    the merged union of two CSR rows: held in shared memory up to 384
+    entries, walked from the two rows beyond.  Tiles are planted at exactly
+    384 and 385 entries, and with interleaved rows (mixed membership bits) on
+    both sides of the cap; every other row keeps its diagonal block."""
+    need_gpu()
+    N, d, B = 32768, 128, 64
+    nb = N // B
+    mask = np.zeros((1, nb, nb), bool)
+    mask[0, np.arange(nb), np.arange(nb)] = True
+    plants = {
+        2: np.arange(0, 300), 3: np.arange(200, 384),            # union 384: list
+        6: np.arange(0, 300), 7: np.arange(200, 385),            # union 385: walk
+        10: np.arange(0, nb, 2), 11: np.arange(1, nb, 2),        # union 512, disjoint: walk
+        14: np.arange(0, 300, 2), 15: np.arange(0, 300, 3),      # union 200, shared entries: list
+    }
+    for q, cols in plants.items():
+        mask[0, q] = False
+        mask[0, q, cols] = True
+    unions = {q: len(set(plants[q]) | set(plants[q + 1])) for q in (2, 6, 10, 14)}
+    assert unions == {2: 384, 6: 385, 10: 512, 14: 200}
+    Q, K, V = rand_qkv(1, N, d, seed=384, qscale=2.0)
+    Os, Ls = gpu_sparse(Q, K, V, mask, B, B)
+    rows = np.concatenate([np.arange(q * B, (q + 1) * B) for q in plants] +
+                          [np.arange(0, 64), np.arange(N - 64, N)])
+    q, k, v = to64(Q[0]), to64(K[0]), to64(V[0])
+    Osr, Lsr = O.sparse_attention_rows(q, k, v, mask[0], B, B, 1.0 / math.sqrt(d), rows)
+    check_attention(Os[0][rows], Osr, "sparse O at the union cap")
+    check_close(to64(Ls)[0, rows], Lsr, LSE_ABS, "sparse LSE at the union cap")
