@@ -130,6 +130,9 @@ SPARSE = [  # heads, N, d, bq, bk, density
     (2, 1000, 128, 128, 128, 0.3), (2, 1000, 128, 64, 64, 0.3), (2, 256, 64, 16, 16, 0.3),
     (2, 1000, 64, 128, 64, 0.25), (2, 1000, 128, 64, 128, 0.4), (2, 600, 128, 16, 64, 0.3),
     (1, 3000, 128, 128, 128, 0.1), (1, 700, 64, 16, 128, 0.5), (2, 333, 128, 128, 16, 0.2),
+    # two 64-row query blocks per tile at d = 64; an odd query-block count,
+    # whose last tile holds one block (its CSR row read directly)
+    (2, 1000, 64, 64, 64, 0.3), (1, 777, 64, 64, 128, 0.35), (2, 1050, 128, 64, 64, 0.3),
 ]
 
 
