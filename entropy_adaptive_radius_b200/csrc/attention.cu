@@ -1303,31 +1303,39 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     const bool use0 = ok && n0 > 0, use1 = ok && n1 > 0;
     const float c0 = use0 ? a0 * inv : 0.f, c1 = use1 ? a1 * inv : 0.f;
     __nv_bfloat16* orow = p.O + (static_cast<size_t>(h) * p.N + (valid_row ? qpos : 0)) * D;
-    // warpgroup w writes output columns [w * D/2, (w + 1) * D/2)
+    // warpgroup w writes output columns [w * D/2, (w + 1) * D/2): all of its
+    // TMEM loads are issued before one wait
+    constexpr int kOutChunks = D / 32;  // 16-column chunks per warpgroup
+    float o0[kOutChunks][16], o1[kOutChunks][16];
 #pragma unroll
-    for (int c = w * (D / 2); c < (w + 1) * (D / 2); c += 16) {
-      float o0[16], o1[16];
-      if (use0) tmem_ld16f(tmem + tl + 2 * BK + c, o0);
-      if (use1) tmem_ld16f(tmem + tl + 2 * BK + D + c, o1);
-      tmem_wait_ld();
-      if (use0) freg_fence<16>(o0);
-      if (use1) freg_fence<16>(o1);
+    for (int k = 0; k < kOutChunks; ++k) {
+      const int c = w * (D / 2) + 16 * k;
+      if (use0) tmem_ld16f(tmem + tl + 2 * BK + c, o0[k]);
+      if (use1) tmem_ld16f(tmem + tl + 2 * BK + D + c, o1[k]);
+    }
+    tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < kOutChunks; ++k) {
+      const int c = w * (D / 2) + 16 * k;
+      if (use0) freg_fence<16>(o0[k]);
+      if (use1) freg_fence<16>(o1[k]);
+      float* o = o0[k];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const float x0 = use0 ? o0[e] * c0 : 0.f;
-        const float x1 = use1 ? o1[e] * c1 : 0.f;
-        o0[e] = x0 + x1;
+        const float x0 = use0 ? o0[k][e] * c0 : 0.f;
+        const float x1 = use1 ? o1[k][e] * c1 : 0.f;
+        o[e] = x0 + x1;
       }
       if (valid_row) {
         uint4 w0, w1;
-        w0.x = pack_bf16(o0[0], o0[1]);
-        w0.y = pack_bf16(o0[2], o0[3]);
-        w0.z = pack_bf16(o0[4], o0[5]);
-        w0.w = pack_bf16(o0[6], o0[7]);
-        w1.x = pack_bf16(o0[8], o0[9]);
-        w1.y = pack_bf16(o0[10], o0[11]);
-        w1.z = pack_bf16(o0[12], o0[13]);
-        w1.w = pack_bf16(o0[14], o0[15]);
+        w0.x = pack_bf16(o[0], o[1]);
+        w0.y = pack_bf16(o[2], o[3]);
+        w0.z = pack_bf16(o[4], o[5]);
+        w0.w = pack_bf16(o[6], o[7]);
+        w1.x = pack_bf16(o[8], o[9]);
+        w1.y = pack_bf16(o[10], o[11]);
+        w1.z = pack_bf16(o[12], o[13]);
+        w1.w = pack_bf16(o[14], o[15]);
         reinterpret_cast<uint4*>(orow + c)[0] = w0;
         reinterpret_cast<uint4*>(orow + c)[1] = w1;
       }
