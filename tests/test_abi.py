@@ -178,3 +178,32 @@ def test_selftest_validation(L):
     assert st(0, None, S0) == INVALID
     assert st(3000, None, S0) == INVALID
     assert st(10, MIS, S0) == INVALID
+
+
+def test_header_compiles_as_c99_and_host_calls_answer(L, tmp_path):
+    """A plain C caller: include/tra.h compiles under -std=c99 -pedantic
+    -Werror, links against libtra.so, and the host-side calls agree with the
+    binding (status strings, workspace size, argument checks)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "abi_host"
+    libdir = os.path.dirname(tra.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c", "abi_host.c"),
+                    "-o", str(exe), "-L", libdir, "-ltra", "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines()
+    kv = {}
+    statuses = []
+    for line in out:
+        key, rest = line.split(" ", 1)
+        if key == "status":
+            statuses.append(rest.split(" ", 1)[1])
+        else:
+            kv[key] = rest
+    assert int(kv["version"]) == L.tra_version()
+    assert statuses == [tra.status_string(s) for s in range(9)] and len(set(statuses)) == 9
+    assert int(kv["workspace"]) == tra.tra_mask_workspace_size(40, (21, 45, 80), 128, 128) > 0
+    assert int(kv["workspace_bad"]) == 0
+    assert int(kv["permute_null"]) == INVALID
