@@ -1247,9 +1247,21 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         };
         // the first half of the keys into registers while this warpgroup's
         // previous PV (which reads P_w) finishes on the tensor cores
+        // (with two 64-key entries the halves are the entries: an unkept one
+        // takes no exponentials, its P is stored as zeros)
+        bool skip_first = false, skip_rest = false;
+        if constexpr (E == 2) {
+          skip_first = !keep_half[0];
+          skip_rest = !keep_half[1];
+        }
         uint32_t first[BK / 4];
+        if (skip_first) {
 #pragma unroll
-        for (int c = 0; c < BK / 4; ++c) first[c] = pair(c);
+          for (int c = 0; c < BK / 4; ++c) first[c] = 0u;
+        } else {
+#pragma unroll
+          for (int c = 0; c < BK / 4; ++c) first[c] = pair(c);
+        }
         if (!wait_prev_pv()) { ok = false; break; }
         rescale_o();
 #pragma unroll
@@ -1257,11 +1269,16 @@ __global__ void __launch_bounds__(kDualThreads, 1)
           st_shared_v4(prow + poff[c8], first[4 * c8], first[4 * c8 + 1], first[4 * c8 + 2],
                        first[4 * c8 + 3]);
         // the rest: computed and stored 8 keys at a time
+        if (skip_rest) {
 #pragma unroll
-        for (int c8 = BK / 16; c8 < BK / 8; ++c8) {
-          const uint32_t a = pair(4 * c8), b = pair(4 * c8 + 1);
-          const uint32_t c = pair(4 * c8 + 2), d = pair(4 * c8 + 3);
-          st_shared_v4(prow + poff[c8], a, b, c, d);
+          for (int c8 = BK / 16; c8 < BK / 8; ++c8) st_shared_v4(prow + poff[c8], 0u, 0u, 0u, 0u);
+        } else {
+#pragma unroll
+          for (int c8 = BK / 16; c8 < BK / 8; ++c8) {
+            const uint32_t a = pair(4 * c8), b = pair(4 * c8 + 1);
+            const uint32_t c = pair(4 * c8 + 2), d = pair(4 * c8 + 3);
+            st_shared_v4(prow + poff[c8], a, b, c, d);
+          }
         }
         const float2 zz = __fadd2_rn(z2[0], z2[1]);
         Z += zz.x + zz.y;
