@@ -616,9 +616,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 // keys is the next two entries of the CTA's key-block list, each loaded into
 // half of a K/V stage (a missing second entry loads rows past N, which read as
 // zeros).  When query blocks have 64 rows the CTA's 128 rows hold two query
-// blocks; its list is the merge of their two CSR rows, and each row masks out
-// the entries its own query block does not keep.  Every role walks that merge
-// itself, in the same order.
+// blocks; its list is the merge of their two CSR rows, and each row leaves
+// out the entries its own query block does not keep.  The prologue counts the
+// merge from bitmaps of both rows (all threads) and, up to 384 entries, writes
+// it to shared memory with membership bits; the softmax reads its entries
+// there (and walks the two rows beyond that size), the producers and issuers
+// walk the merge themselves, in the same order.  With two 64-key entries a
+// warp (64 rows of one query block) keeps each half of a super-block whole or
+// not at all, except in the sequence's last key block: an unkept half is left
+// out of the row max and takes no exponentials (its P is stored as zeros).
 // ---------------------------------------------------------------------------
 
 constexpr int kDualThreads = 384;  // 12 warps
