@@ -20,8 +20,7 @@ section names follow the Japanese page):
     that turns the token mask into a block-sparse mask; entropy reused across
     denoising steps.
 
-Readings taken where the pages leave a step open (each is listed, with its
-reason, in the design notes of the repository):
+Readings taken where the pages leave a step open:
   R1 scores s_ij = q_i . k_j / sqrt(d); natural logarithm.
   R2 entropy over all N keys of the same head.
   R3 tile-major order: tiles ordered frame-tile, tile-row, tile-col; inside a
