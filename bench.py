@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -409,8 +410,9 @@ def gpu_arm(args, rank, world, local):
     if tra.tra_get_device_error() != 0:
         raise RuntimeError("device-side wait timed out during warm-up")
 
-    sampler = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-                           if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/tra_clocks_{rank}.csv")
+    clocks_csv = (args.clocks_csv.replace("{rank}", str(rank)) if args.clocks_csv
+                  else os.path.join(tempfile.gettempdir(), f"tra_clocks_rank{rank}_{os.getpid()}.csv"))
+    sampler = ClockSampler(local, clocks_csv)
     rec = []
     pipe.launches = 0
     if world > 1:
@@ -994,6 +996,9 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="tra", choices=["tra", "reference"])
+    ap.add_argument("--clocks-csv", default=None,
+                    help="where the nvidia-smi clock samples of the timed region go "
+                         "({rank} is replaced by the rank); default: a temporary file")
     args = ap.parse_args()
     rank, world, local = dist_env()
     if args.case is not None:
