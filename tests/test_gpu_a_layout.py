@@ -108,3 +108,31 @@ def test_budget_radius(wl, tau):
         np.testing.assert_allclose(rg[h][fin], ref[fin], rtol=2e-6, atol=0)
         assert np.array_equal(np.isinf(rg[h]), np.isinf(ref))
     assert rg[0, 0] == np.inf and rg[0, 1] == 0.0
+
+
+@pytest.mark.parametrize("grid,tau,gamma", [((1, 8, 8), 0.05, 0.3), ((5, 8, 12), 0.05, 0.0),
+                                            ((5, 8, 12), 0.05, 20.0), ((5, 8, 12), 0.0, 0.3),
+                                            ((7, 4, 4), 3.0, 1.0)])
+def test_budget_radius_parameter_corners(grid, tau, gamma):
+    """One frame (S = 1); gamma = 0 (phi = 1, S = F); a steep decay (phi(1) ~
+    2e-9); tau = 0 (every radius 0); a grid of a single tile per frame."""
+    need_gpu()
+    F, Hh, W = grid
+    N = F * Hh * W
+    heads = 3
+    tile = (1, 4, 4)
+    Hs = inputs.synthetic_entropy(heads, N, 11, math.log(N) - 2.0, math.log(N))
+    pi = O.tile_major_order(F, Hh, W, tile)
+    t_tm = O.token_coords(F, Hh, W)[pi][:, 2]
+    Hd = torch.from_numpy(Hs).cuda()
+    r = torch.empty_like(Hd)
+    phi = torch.empty(F, dtype=torch.float32, device="cuda")
+    tra.tra_budget_radius(Hd, r, grid, tau, gamma, tile, phi_out=phi)
+    tau32, gamma32 = float(np.float32(tau)), float(np.float32(gamma))
+    np.testing.assert_allclose(phi.cpu().numpy(), O.phi(np.arange(F), gamma32), rtol=1e-7, atol=0)
+    rg = r.cpu().numpy().astype(np.float64)
+    for h in range(heads):
+        ref = O.radius(Hs[h].astype(np.float64), t_tm, tau32, gamma32, F, N)
+        np.testing.assert_allclose(rg[h], ref, rtol=2e-6, atol=0)
+    if tau == 0.0:
+        assert not rg.any()

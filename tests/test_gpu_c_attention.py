@@ -245,3 +245,33 @@ def test_union_list_and_walk_fallback_at_the_cap():
     Osr, Lsr = O.sparse_attention_rows(q, k, v, mask[0], B, B, 1.0 / math.sqrt(d), rows)
     check_attention(Os[0][rows], Osr, "sparse O at the union cap")
     check_close(to64(Ls)[0, rows], Lsr, LSE_ABS, "sparse LSE at the union cap")
+
+
+@pytest.mark.parametrize("scale", [0.03, 0.4])
+def test_dense_and_sparse_with_a_given_scale(scale):
+    """The softmax scale is an argument of both calls (the default is
+    1/sqrt(d)); a small scale flattens the rows, a large one sharpens them."""
+    need_gpu()
+    heads, N, d, B = 2, 700, 128, 64
+    Q, K, V = rand_qkv(heads, N, d, seed=int(scale * 1000))
+    Qd, Kd, Vd = (t.cuda() for t in (Q, K, V))
+    O_ = torch.empty_like(Qd)
+    H = torch.empty(heads, N, dtype=torch.float32, device="cuda")
+    L = torch.empty_like(H)
+    tra.tra_dense_attn_entropy(Qd, Kd, Vd, O_, H, L, scale=scale)
+    assert tra.tra_get_device_error() == 0
+    Or, Hr, Lr = O.dense_attention_entropy(to64(Q), to64(K), to64(V), scale)
+    check_attention(O_, Or, f"dense O scale {scale}")
+    check_close(H, Hr, H_ABS, f"H scale {scale}")
+    check_close(L, Lr, LSE_ABS, f"LSE scale {scale}")
+    nb = -(-N // B)
+    mask = inputs.synthetic_block_mask(heads, nb, nb, seed=7, density=0.3)
+    rp, ci = inputs.csr_from_block_mask(mask)
+    Os = torch.empty_like(Qd)
+    Ls = torch.empty_like(H)
+    tra.tra_block_sparse_attn(Qd, Kd, Vd, Os, torch.from_numpy(rp.ravel()).cuda(),
+                              torch.from_numpy(ci).cuda(), B, B, lse=Ls, scale=scale)
+    assert tra.tra_get_device_error() == 0
+    Osr, Lsr = O.sparse_attention(to64(Q), to64(K), to64(V), mask, B, B, scale)
+    check_attention(Os, Osr, f"sparse O scale {scale}")
+    check_close(Ls, Lsr, LSE_ABS, f"sparse LSE scale {scale}")
