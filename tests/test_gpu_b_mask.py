@@ -187,3 +187,44 @@ def test_mask_frame_count_extremes(grid, tile, bq, bk, vote):
     assert np.array_equal(rp, rp_ref)
     assert np.array_equal(ci[:nnz], ci_ref)
     assert 0.0 < nnz / (2 * (-(-N // bq)) * (-(-N // bk))) < 1.0
+
+
+@pytest.mark.parametrize("vote,hi", [(257, 3.0), (40, 2.5)])
+def test_mask_with_empty_rows_drives_attention(vote, hi):
+    """A vote threshold above |qb| * |kb| keeps nothing (nnz = 0, every CSR row
+    empty); one above the self votes with small radii empties some rows.  The
+    CSR matches the oracle bit for bit, and the block-sparse call over it gives
+    O = 0 and LSE = -inf on the empty rows and the oracle's attention on the
+    others."""
+    need_gpu()
+    grid, tile, B = (4, 8, 8), (1, 4, 4), 16
+    F, H, W = grid
+    N = F * H * W
+    heads = 2
+    r = inputs.synthetic_radius(heads, N, seed=vote, lo=0.2, hi=hi, special=False)
+    phi = O.phi(np.arange(F), 0.4).astype(np.float32)
+    rp, ci, nnz = run_mask(r, phi, grid, tile, B, B, vote)
+    rp_ref, ci_ref, masks = oracle_csr(r, phi, grid, tile, B, B, vote)
+    assert nnz == len(ci_ref) and np.array_equal(rp, rp_ref) and np.array_equal(ci[:nnz], ci_ref)
+    empty = ~masks.any(axis=2)
+    if vote > B * B:
+        assert nnz == 0 and empty.all()
+    else:
+        assert empty.any() and not empty.all()
+    g = torch.Generator().manual_seed(vote)
+    Q, K, V = (torch.randn(heads, N, 64, generator=g).to(torch.bfloat16) for _ in range(3))
+    Os = torch.full((heads, N, 64), 3.0, dtype=torch.bfloat16, device="cuda")
+    Ls = torch.empty(heads, N, dtype=torch.float32, device="cuda")
+    ci_d = torch.from_numpy(ci[:max(nnz, 1)] if nnz else np.zeros(1, np.int32)).cuda()
+    tra.tra_block_sparse_attn(Q.cuda(), K.cuda(), V.cuda(), Os, torch.from_numpy(rp).cuda(), ci_d,
+                              B, B, lse=Ls)
+    assert tra.tra_get_device_error() == 0
+    Or, Lr = O.sparse_attention(Q.double().numpy(), K.double().numpy(), V.double().numpy(), masks,
+                                B, B, 1.0 / math.sqrt(64))
+    rows_empty = np.repeat(empty, B, axis=1)[:, :N]
+    Osn, Lsn = Os.float().cpu().numpy(), Ls.cpu().numpy()
+    assert (Osn[rows_empty] == 0).all() and np.isneginf(Lsn[rows_empty]).all()
+    assert np.abs(Osn - Or).max() <= 2e-2 and np.abs(Osn - Or).mean() <= 2e-3
+    keep = ~rows_empty
+    if keep.any():
+        assert np.abs(Lsn[keep] - Lr[keep]).max() <= 1e-3
