@@ -70,8 +70,10 @@ def margin(Hs, tau, c):
     return worst
 
 
-@pytest.mark.parametrize("refresh", ["entropy", "dense"])
-def test_reuse_loop_matches_oracle_schedule(refresh):
+@pytest.mark.parametrize("refresh,dtype", [("entropy", "bf16"), ("dense", "bf16"), ("entropy", "f32")])
+def test_reuse_loop_matches_oracle_schedule(refresh, dtype):
+    """dtype f32 hands the layer the same (bf16-valued) inputs as float32
+    tensors: its permute then rounds them to bf16, exactly."""
     need_gpu()
     steps = make_steps(seed=5)
     policy = ReusePolicy(warmup=1, refresh_every=2, refresh=refresh)
@@ -98,6 +100,8 @@ def test_reuse_loop_matches_oracle_schedule(refresh):
                      block_k=BK, policy=policy)
     nqb = -(-N // BQ)
     for k, (Q, K, V) in enumerate(steps):
+        if dtype == "f32":
+            Q, K, V = Q.float(), K.float(), V.float()
         Og = layer(Q.cuda(), K.cuda(), V.cuda())
         assert tra.tra_get_device_error() == 0
         check_attention(Og, O.inverse_permute(outs[k], pi), f"step {k} ({plan[k]})")
