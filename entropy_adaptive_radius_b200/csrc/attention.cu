@@ -1382,19 +1382,31 @@ __global__ void __launch_bounds__(kDualThreads, 1)
 // Entropy-only pass: H and LSE of every query over all N keys, without the
 // PV product or the output (an entropy refresh that needs no dense output).
 //
-// Same split as the two-warpgroup kernel: warpgroup w takes key blocks
-// j = w, w + 2, ...; with no output accumulator each warpgroup has two TMEM
-// score tiles (S_{w,0}, S_{w,1}), so the MMA warp can run two of its QK
-// products ahead.  K has a 4-stage ring.  Per score the softmax does one
-// packed FMA (x = s * scale * log2 e - m), one ex2 and half of a packed add
-// (Z) and of a packed FMA (A): the MUFU unit bounds it, the tensor cores run
-// at half their dense-pass load.  Warps: 0..7 softmax, 8 Q/K producer (and
-// tensor-memory allocation), 9 MMA.
+// With no output accumulator the 512 TMEM columns hold four score tiles, one
+// per softmax warpgroup: warpgroup w takes key blocks j = w, w + 4, ... and
+// reads its tile in two halves of 64 scores, so that four warpgroups fit the
+// register file (setmaxnreg: 104 per softmax thread, 64 for the producer /
+// MMA warpgroup) and each scheduler has four softmax warps to issue from.  K
+// has a 4-stage ring.  Per score the softmax does one packed FMA
+// (x = s * scale * log2 e - m), one ex2 and half of a packed add (Z) and of a
+// packed FMA (A): the MUFU unit bounds it, the tensor cores run at half their
+// dense-pass load.  The four warpgroups' (m, Z, A) are merged exactly at the
+// end.  Warps: 0..15 softmax, 16 Q/K producer (and tensor-memory allocation),
+// 17 MMA, 18 and 19 idle (they complete the fifth warpgroup).
 // ---------------------------------------------------------------------------
 
-constexpr int kEntThreads = 320;  // 10 warps
-constexpr int kEntKWarp = 8;
-constexpr int kEntMmaWarp = 9;
+constexpr int kEntThreads = 640;  // 20 warps
+constexpr int kEntWarpgroups = 4; // softmax warpgroups (warps 0..15)
+constexpr int kEntKWarp = 16;
+constexpr int kEntMmaWarp = 17;
+// Registers: launched at 96 per thread (640 x 96 = 61440); the softmax
+// warpgroups take 104, the producer / MMA warpgroup gives back to 64:
+// 4 x 128 x 104 + 128 x 64 = 61440.
+constexpr int kEntRegsLaunch = 96;
+constexpr int kEntRegsSoftmax = 104;
+constexpr int kEntRegsOther = 64;
+static_assert(kEntWarpgroups * 128 * kEntRegsSoftmax + 128 * kEntRegsOther ==
+                  kEntThreads * kEntRegsLaunch, "register split");
 
 template <int D>
 struct EntCfg {
@@ -1405,14 +1417,14 @@ struct EntCfg {
   static constexpr int KV_BYTES = BK * D * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_ST = OFF_K + NS * KV_BYTES;  // merge statistics, 2 x 3 x 128 fp32
-  static constexpr int OFF_BAR = OFF_ST + 2 * 3 * BM * 4;
+  static constexpr int OFF_ST = OFF_K + NS * KV_BYTES;  // merge statistics, 4 x 3 x 128 fp32
+  static constexpr int OFF_BAR = OFF_ST + kEntWarpgroups * 3 * BM * 4;
   static constexpr int NUM_BARS = 1 + 2 * NS + 8 + 1;
   static constexpr int OFF_MISC = OFF_BAR + 256;
   static constexpr int USED = OFF_MISC + 64;
   static constexpr int SMEM = (USED < 120 * 1024 ? 120 * 1024 : USED) + 1024;
-  static constexpr int TMEM_COLS = 512;  // S_{0,0}, S_{0,1}, S_{1,0}, S_{1,1}
-  static_assert(4 * BK <= TMEM_COLS, "tensor memory");
+  static constexpr int TMEM_COLS = 512;  // one 128-column score tile per warpgroup
+  static_assert(kEntWarpgroups * BK <= TMEM_COLS, "tensor memory");
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(NUM_BARS * 8 <= 256, "barrier area");
 };
@@ -1424,6 +1436,7 @@ __global__ void __launch_bounds__(kEntThreads, 1)
   using C = EntCfg<D>;
   constexpr int NS = C::NS;
   constexpr int BK = C::BK;
+  constexpr int WG = kEntWarpgroups;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -1434,8 +1447,8 @@ __global__ void __launch_bounds__(kEntThreads, 1)
   const uint32_t bar_q = bars;
   auto k_full = [&](int s) { return bars + 8u * (1 + s); };
   auto k_empty = [&](int s) { return bars + 8u * (1 + NS + s); };
-  auto s_full = [&](int t) { return bars + 8u * (1 + 2 * NS + t); };   // t = 2 w + buffer
-  auto s_free = [&](int t) { return bars + 8u * (5 + 2 * NS + t); };
+  auto s_full = [&](int w) { return bars + 8u * (1 + 2 * NS + w); };
+  auto s_free = [&](int w) { return bars + 8u * (5 + 2 * NS + w); };
   const uint32_t drain_bar = bars + 8u * (9 + 2 * NS);
   volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   volatile int* abort = misc + 1;
@@ -1451,9 +1464,9 @@ __global__ void __launch_bounds__(kEntThreads, 1)
       mbar_init(k_full(s), 1);
       mbar_init(k_empty(s), 1);
     }
-    for (int t = 0; t < 4; ++t) {
-      mbar_init(s_full(t), 1);
-      mbar_init(s_free(t), 128);
+    for (int w = 0; w < WG; ++w) {
+      mbar_init(s_full(w), 1);
+      mbar_init(s_free(w), 128);
     }
     mbar_init(drain_bar, 1);
     fence_barrier_init();
@@ -1471,6 +1484,9 @@ __global__ void __launch_bounds__(kEntThreads, 1)
   tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
 
+  if (warp >= 4 * WG) {
+  // the producer / MMA warpgroup gives registers back (all four warps)
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kEntRegsOther));
   if (warp == kEntKWarp) {
     // ===================================================== Q / K producer
     if (lane == 0) {
@@ -1495,16 +1511,17 @@ __global__ void __launch_bounds__(kEntThreads, 1)
     }
   } else if (warp == kEntMmaWarp) {
     // ===================================================== MMA issuer (QK only, in block order)
+    // block j goes to warpgroup j mod 4 and its score tile S_{j mod 4}
     if (lane == 0) {
       constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BK, 0, 0);
       bool ok = mbar_wait(bar_q, 0, abort, p.err, kErrWaitQ);
       for (int j = 0; ok && j < nblk; ++j) {
-        const int s = j % NS, w = j & 1, i = j >> 1, t = 2 * w + (i & 1), u = i >> 1;
+        const int s = j % NS, w = j % WG, u = j / WG;
         ok = mbar_wait(k_full(s), (j / NS) & 1, abort, p.err, kErrWaitKFull) &&
-             mbar_wait(s_free(t), (u & 1) ^ 1u, abort, p.err, kErrWaitSFree);
+             mbar_wait(s_free(w), (u & 1) ^ 1u, abort, p.err, kErrWaitSFree);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t tS = tmem + t * BK;
+        const uint32_t tS = tmem + w * BK;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint64_t a = smem_desc_sw128(sQ + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024);
@@ -1513,100 +1530,112 @@ __global__ void __launch_bounds__(kEntThreads, 1)
           mma_bf16_ss(tS, a, bd, kIdescQK, k > 0 ? 1u : 0u);
         }
         mma_commit(k_empty(s));
-        mma_commit(s_full(t));
+        mma_commit(s_full(w));
       }
       if (!ok) {
         mma_commit(drain_bar);
         drain_wait(drain_bar, 0);
       }
     }
-  } else if (warp < 8) {
-    // ===================================================== softmax statistics (warps 0..7)
+  }
+  } else {
+    // ===================================================== softmax statistics (warps 0..15)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEntRegsSoftmax));
     const int w = warp >> 2;
     const int row = tid & 127;
     const uint32_t tl = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + tl + w * BK;
     const int qpos = qt * BM + row;
-    const int nmine = (nblk + 1 - w) >> 1;
+    const int nmine = nblk > w ? (nblk - 1 - w) / WG + 1 : 0;
     float m_ref = -INFINITY, Z = 0.f, A = 0.f;
     bool ok = true;
-    float sv[BK];
     for (int i = 0; i < nmine; ++i) {
-      const int j = 2 * i + w;
-      const int t = 2 * w + (i & 1), u = i >> 1;
-      ok = mbar_wait(s_full(t), u & 1, abort, p.err, kErrWaitSFull);
+      const int j = WG * i + w;
+      ok = mbar_wait(s_full(w), i & 1, abort, p.err, kErrWaitSFull);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < BK / 32; ++c) tmem_ld32f(tmem + tl + t * BK + c * 32, sv + c * 32);
-      tmem_wait_ld();
-      freg_fence<BK>(sv);
-      tc_fence_before();
-      mbar_arrive(s_free(t));
       const int nvalid = min(BK, p.N - j * BK);  // keys past N (zero rows) are excluded
-      if (nvalid < BK) {
+      // the score row in two halves of 64 (registers for four warpgroups);
+      // S_w is released once both halves are in registers
 #pragma unroll
-        for (int c = 0; c < BK; ++c) sv[c] = c < nvalid ? sv[c] : -1e30f;
-      }
-      {
-        float mx[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          mx[q] = fmax3(sv[q], sv[16 + q], sv[32 + q]);
-          mx[q] = fmax3(mx[q], sv[48 + q], sv[64 + q]);
-          mx[q] = fmax3(mx[q], sv[80 + q], sv[96 + q]);
-          mx[q] = fmaxf(mx[q], sv[112 + q]);
+      for (int hh = 0; hh < 2; ++hh) {
+        float sv[BK / 2];
+        tmem_ld32f(tS + hh * (BK / 2), sv);
+        tmem_ld32f(tS + hh * (BK / 2) + 32, sv + 32);
+        tmem_wait_ld();
+        freg_fence<BK / 2>(sv);
+        if (hh == 1) {
+          tc_fence_before();
+          mbar_arrive(s_free(w));
         }
+        if (nvalid < BK) {
 #pragma unroll
-        for (int q = 0; q < 5; ++q) mx[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
-        const float bmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[15])) *
-                           p.scale_log2;
-        const float m_new = fmaxf(m_ref, bmax);
-        if (m_new > m_ref + kRescaleLog2) {
-          if (m_ref != -INFINITY) {
-            const float alpha = ex2_approx(m_ref - m_new);
-            A = alpha * (A + (m_ref - m_new) * Z);
-            Z *= alpha;
+          for (int c = 0; c < BK / 2; ++c) sv[c] = hh * (BK / 2) + c < nvalid ? sv[c] : -1e30f;
+        }
+        {
+          float mx[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            mx[q] = fmax3(sv[q], sv[16 + q], sv[32 + q]);
+            mx[q] = fmaxf(mx[q], sv[48 + q]);
           }
-          m_ref = m_new;
+#pragma unroll
+          for (int q = 0; q < 5; ++q) mx[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
+          const float bmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[15])) *
+                             p.scale_log2;
+          const float m_new = fmaxf(m_ref, bmax);
+          if (m_new > m_ref + kRescaleLog2) {
+            if (m_ref != -INFINITY) {
+              const float alpha = ex2_approx(m_ref - m_new);
+              A = alpha * (A + (m_ref - m_new) * Z);
+              Z *= alpha;
+            }
+            m_ref = m_new;
+          }
         }
-      }
-      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-      const float2 nm2 = make_float2(-m_ref, -m_ref);
-      float2 z2[4], a2[4];
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(-m_ref, -m_ref);
+        float2 z2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        z2[q] = make_float2(0.f, 0.f);
-        a2[q] = make_float2(0.f, 0.f);
+        for (int c = 0; c < BK / 4; ++c) {
+          const float2 x = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nm2);
+          const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          z2[c & 1] = __fadd2_rn(z2[c & 1], pr);
+          a2[c & 1] = __ffma2_rn(pr, x, a2[c & 1]);
+        }
+        const float2 zz = __fadd2_rn(z2[0], z2[1]);
+        const float2 aa = __fadd2_rn(a2[0], a2[1]);
+        Z += zz.x + zz.y;
+        A += aa.x + aa.y;
       }
-#pragma unroll
-      for (int c = 0; c < BK / 2; ++c) {
-        const float2 x = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nm2);
-        const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-        z2[c & 3] = __fadd2_rn(z2[c & 3], pr);
-        a2[c & 3] = __ffma2_rn(pr, x, a2[c & 3]);
-      }
-      const float2 zz = __fadd2_rn(__fadd2_rn(z2[0], z2[1]), __fadd2_rn(z2[2], z2[3]));
-      const float2 aa = __fadd2_rn(__fadd2_rn(a2[0], a2[1]), __fadd2_rn(a2[2], a2[3]));
-      Z += zz.x + zz.y;
-      A += aa.x + aa.y;
     }
-    // ---- merge the two warpgroups' statistics; warpgroup 0 writes H and LSE
+    // ---- merge the four warpgroups' statistics; warpgroup 0 writes H and LSE
     float* st = reinterpret_cast<float*>(smem + C::OFF_ST);
     st[(w * 3 + 0) * BM + row] = ok ? m_ref : -INFINITY;
     st[(w * 3 + 1) * BM + row] = ok ? Z : 0.f;
     st[(w * 3 + 2) * BM + row] = ok ? A : 0.f;
-    named_barrier_sync(1, 256);
+    named_barrier_sync(1, WG * 128);
     if (w == 0 && qpos < p.N) {
-      const float m0 = st[0 * BM + row], Z0 = st[1 * BM + row], A0 = st[2 * BM + row];
-      const float m1 = st[3 * BM + row], Z1 = st[4 * BM + row], A1 = st[5 * BM + row];
-      const float m = fmaxf(m0, m1);
-      const float a0 = (m0 == -INFINITY) ? 0.f : ex2_approx(m0 - m);
-      const float a1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - m);
-      const float Zt = a0 * Z0 + a1 * Z1;
-      float At = 0.f;
-      if (a0 > 0.f) At += a0 * (A0 + (m0 - m) * Z0);
-      if (a1 > 0.f) At += a1 * (A1 + (m1 - m) * Z1);
+      float mw[WG], Zw[WG], Aw[WG];
+      float m = -INFINITY;
+#pragma unroll
+      for (int g = 0; g < WG; ++g) {
+        mw[g] = st[(g * 3 + 0) * BM + row];
+        Zw[g] = st[(g * 3 + 1) * BM + row];
+        Aw[g] = st[(g * 3 + 2) * BM + row];
+        m = fmaxf(m, mw[g]);
+      }
+      float Zt = 0.f, At = 0.f;
+#pragma unroll
+      for (int g = 0; g < WG; ++g) {
+        const float ag = (mw[g] == -INFINITY) ? 0.f : ex2_approx(mw[g] - m);
+        if (ag > 0.f) {
+          Zt += ag * Zw[g];
+          At += ag * (Aw[g] + (mw[g] - m) * Zw[g]);
+        }
+      }
       const size_t idx = static_cast<size_t>(h) * p.N + qpos;
       p.H[idx] = Zt > 0.f ? logf(Zt) - kLn2 * (At / Zt) : NAN;
       if (p.lse != nullptr) p.lse[idx] = Zt > 0.f ? kLn2 * (m + log2f(Zt)) : -INFINITY;
@@ -1688,7 +1717,12 @@ cudaError_t launch_entropy(const AttnArgs& a, const Params& prm, cudaStream_t st
   if (!make_map(&mq, a.Q, D, a.N, a.heads, BM) || !make_map(&mk, a.K, D, a.N, a.heads, 128))
     return cudaErrorInvalidValue;
   auto kern = entropy_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  // the setmaxnreg split assumes the launch allocation: refuse any other
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, kern);
+  if (e != cudaSuccess) return e;
+  if (attr.numRegs != kEntRegsLaunch) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const dim3 grid((a.N + BM - 1) / BM, a.heads);
   kern<<<grid, kEntThreads, C::SMEM, stream>>>(mq, mk, prm);
