@@ -17,11 +17,17 @@
 //  2. votes: one CTA per (head, query block).  Each CTA bounds, for every key
 //     frame, the union of its queries' disks by a box; a key block whose
 //     per-frame boxes miss those boxes has no votes and is pruned (lanes over
-//     key blocks).  Survivors are counted exactly (lanes over queries): for a
-//     query and a key row the number of keys inside the disk is the overlap of
-//     [x_lo, x_hi] with [x_q - s, x_q + s], s = isqrt(floor(R2) - dy^2); with a
-//     vote threshold of 1 an existence test replaces the count.  Counting stops
-//     once the threshold is reached (only "votes >= threshold" is needed).
+//     key blocks).  A survivor is then rejected when no query's disk meets any
+//     of its per-frame boxes.  With a vote threshold of 1 and the disk distance
+//     the block's complete rectangles (runs of rows of one frame with the same
+//     x interval, every lattice position a key) decide exactly: the nearest
+//     point of such a rectangle to a query is one of its keys, so one
+//     dx^2 + dy^2 test per (query, rectangle) answers.  Otherwise survivors are
+//     counted exactly (lanes over queries): for a query and a key row the
+//     number of keys inside the disk is the overlap of [x_lo, x_hi] with
+//     [x_q - s, x_q + s], s = isqrt(floor(R2) - dy^2); with a vote threshold
+//     of 1 an existence test replaces the count.  Counting stops once the
+//     threshold is reached (only "votes >= threshold" is needed).
 //  3. scan: exclusive prefix sum of the per-row kept counts -> row_ptr, nnz.
 //  4. compact: kept bits -> ascending col_idx.
 //
