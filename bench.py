@@ -483,7 +483,14 @@ def gpu_arm(args, rank, world, local):
             perm_ms.append(e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]))
             sparse_ms.append(e[1].elapsed_time(e[2]))
     ms_step = elapsed_ms / args.steps
-    value = world * fl_step / (ms_step * 1e-3) / 1e12
+    # whole-job work: every rank calibrates its own tau on its own inputs, so
+    # the ranks' kept work differs a little; the job's flops are their sum
+    fl_job = fl_step
+    if world > 1:
+        t = torch.tensor([fl_step], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        fl_job = float(t.item())
+    value = fl_job / (ms_step * 1e-3) / 1e12
     d_ms, s_ms = statistics.mean(dense_ms), statistics.mean(sparse_ms)
     peaks, peak_kind = load_peaks()
     dense_tf = fl_dense / (d_ms * 1e-3) / 1e12
@@ -526,7 +533,7 @@ def gpu_arm(args, rank, world, local):
             "unamortised_ratio_to_1_call": round((max(0.0, entropy_ms) + mask_total) / s_ms, 4),
             "sparse_calls": calls},
         "tile_major_resident": {"ms_per_step": round(res_ms, 3),
-                                "value": round(world * fl_step / (res_ms * 1e-3) / 1e12, 3),
+                                "value": round(fl_job / (res_ms * 1e-3) / 1e12, 3),
                                 "unit": UNIT, "note": "same step, tokens kept in tile-major order "
                                 "between calls: no per-call permutes"},
         "roofline": roofline, "roofline_sparse": roofline_sparse, "roofline_permute": roofline_permute,
@@ -535,7 +542,7 @@ def gpu_arm(args, rank, world, local):
 
     # ---- end to end: host (pinned) inputs copied in, O copied back, every call
     e2e = e2e_run(pipe, host, dev, calls, args, device, world)
-    out["e2e"] = {"value": round(world * fl_step / (e2e["ms"] * 1e-3) / 1e12, 3), "unit": UNIT,
+    out["e2e"] = {"value": round(fl_job / (e2e["ms"] * 1e-3) / 1e12, 3), "unit": UNIT,
                   "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                   "ms_per_step": round(e2e["ms"], 3)}
     if rank == 0 and world == 1:
