@@ -789,7 +789,8 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       misc[2] = (n[0] + E - 1) / E;
       misc[3] = st[0]; misc[4] = n[0]; misc[5] = st[1]; misc[6] = n[1];
       misc[7] = 0;
-      misc[8] = 0;  // 1: the merged list is in shared memory
+      misc[8] = 0;   // 1: the merged list is in shared memory
+      misc[10] = 0;  // malformed rows (bit 0: A, bit 1: B)
     }
   }
   if (warp == kDualKWarp) {
@@ -810,67 +811,99 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       // stored; each holds 262144 bits, the largest nKB).  A list of at most
       // kUnionCap entries is then written out in order, with membership bits,
       // so the softmax reads its entries instead of walking the two rows.
+      // The same pass checks that each row is strictly ascending within
+      // [0, nKB): the softmax and the producers would otherwise disagree on
+      // the list, and one malformed row would spoil the other block's output.
+      // A malformed row is skipped (and reported), like a bad start or length.
       static_assert(C::P_BYTES * 8 >= (1 << 24) / 64, "key-block bitmap");
-      const int na = misc[4], nb = misc[6];
       const int* a = p.col_idx + misc[3];
       const int* b = p.col_idx + misc[5];
       uint32_t* bma = reinterpret_cast<uint32_t*>(smem + C::OFF_P);
       uint32_t* bmb = reinterpret_cast<uint32_t*>(smem + C::OFF_P + C::P_BYTES);
       const int nw = (p.nkb + 31) >> 5;
-      for (int i = tid; i < nw; i += kDualThreads) {
-        bma[i] = 0u;
-        bmb[i] = 0u;
-      }
-      __syncthreads();
-      for (int i = tid; i < na; i += kDualThreads) {
-        const int kb = __ldg(a + i);
-        if (kb >= 0 && kb < p.nkb) atomicOr(bma + (kb >> 5), 1u << (kb & 31));
-      }
-      __syncthreads();
-      int both = 0;
-      for (int i = tid; i < nb; i += kDualThreads) {
-        const int kb = __ldg(b + i);
-        if (kb >= 0 && kb < p.nkb) {
-          both += static_cast<int>((bma[kb >> 5] >> (kb & 31)) & 1u);
-          atomicOr(bmb + (kb >> 5), 1u << (kb & 31));
+      // bitmaps of rows A (na entries) and B (nb entries) and their common
+      // entries (misc[7]); returns the malformed-row bits (misc[10])
+      auto build_bitmaps = [&](int na, int nb) -> uint32_t {
+        for (int i = tid; i < nw; i += kDualThreads) {
+          bma[i] = 0u;
+          bmb[i] = 0u;
         }
+        __syncthreads();
+        uint32_t bad = 0u;
+        for (int i = tid; i < na; i += kDualThreads) {
+          const int kb = __ldg(a + i);
+          if (kb < 0 || kb >= p.nkb || (i + 1 < na && __ldg(a + i + 1) <= kb)) bad |= 1u;
+          else atomicOr(bma + (kb >> 5), 1u << (kb & 31));
+        }
+        __syncthreads();
+        int both = 0;
+        for (int i = tid; i < nb; i += kDualThreads) {
+          const int kb = __ldg(b + i);
+          if (kb < 0 || kb >= p.nkb || (i + 1 < nb && __ldg(b + i + 1) <= kb)) {
+            bad |= 2u;
+          } else {
+            both += static_cast<int>((bma[kb >> 5] >> (kb & 31)) & 1u);
+            atomicOr(bmb + (kb >> 5), 1u << (kb & 31));
+          }
+        }
+        both = __reduce_add_sync(0xffffffffu, both);
+        bad = __reduce_or_sync(0xffffffffu, bad);
+        if (lane == 0 && both > 0) atomicAdd(const_cast<int*>(misc + 7), both);
+        if (lane == 0 && bad != 0u) atomicOr(const_cast<int*>(misc + 10), static_cast<int>(bad));
+        __syncthreads();
+        return static_cast<uint32_t>(misc[10]);
+      };
+      const uint32_t bad = build_bitmaps(misc[4], misc[6]);
+      if (bad != 0u) {
+        __syncthreads();  // every thread has read misc[10]
+        if (tid == 0) {
+          if (bad & 1u) misc[4] = 0;
+          if (bad & 2u) misc[6] = 0;
+          misc[2] = (misc[4] + E - 1) / E;  // the tile's one remaining row (or none)
+          misc[7] = 0;
+          misc[10] = 0;
+          if (p.err) atomicCAS(p.err, 0, kErrBadCsr);
+        }
+        __syncthreads();
+        // A skipped, B kept: B alone goes through the merged list (its
+        // entries carry B's membership bit)
+        if (misc[6] > 0) build_bitmaps(0, misc[6]);
       }
-      both = __reduce_add_sync(0xffffffffu, both);
-      if (lane == 0 && both > 0) atomicAdd(const_cast<int*>(misc + 7), both);
-      __syncthreads();
-      const int ulen = na + nb - misc[7];
-      if (tid == 0) {
-        misc[2] = (ulen + E - 1) / E;
-        misc[9] = ulen;
-      }
-      if (ulen <= C::kUnionCap && warp == 0) {
-        // warp 0 writes the set bits of A | B in ascending order, 32 words a round
-        uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
-        int run = 0;
-        for (int base = 0; base < nw; base += 32) {
-          const int wd = base + lane;
-          const uint32_t wa = wd < nw ? bma[wd] : 0u, wb = wd < nw ? bmb[wd] : 0u;
-          uint32_t word = wa | wb;
-          const int cnt = __popc(word);
-          int incl = cnt;
+      if (misc[6] > 0) {
+        const int ulen = misc[4] + misc[6] - misc[7];
+        if (tid == 0) {
+          misc[2] = (ulen + E - 1) / E;
+          misc[9] = ulen;
+        }
+        if (ulen <= C::kUnionCap && warp == 0) {
+          // warp 0 writes the set bits of A | B in ascending order, 32 words a round
+          uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
+          int run = 0;
+          for (int base = 0; base < nw; base += 32) {
+            const int wd = base + lane;
+            const uint32_t wa = wd < nw ? bma[wd] : 0u, wb = wd < nw ? bmb[wd] : 0u;
+            uint32_t word = wa | wb;
+            const int cnt = __popc(word);
+            int incl = cnt;
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
+            for (int o = 1; o < 32; o <<= 1) {
+              const int v = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += v;
+            }
+            int pos = run + incl - cnt;
+            while (word) {
+              const int bit = __ffs(word) - 1;
+              word &= word - 1;
+              const uint32_t mem = ((wa >> bit) & 1u) | (((wb >> bit) & 1u) << 1);
+              if (pos < C::kUnionCap) list[pos] = static_cast<uint32_t>(wd * 32 + bit) | (mem << 30);
+              ++pos;
+            }
+            run += __shfl_sync(0xffffffffu, incl, 31);
           }
-          int pos = run + incl - cnt;
-          while (word) {
-            const int bit = __ffs(word) - 1;
-            word &= word - 1;
-            const uint32_t mem = ((wa >> bit) & 1u) | (((wb >> bit) & 1u) << 1);
-            if (pos < C::kUnionCap) list[pos] = static_cast<uint32_t>(wd * 32 + bit) | (mem << 30);
-            ++pos;
-          }
-          run += __shfl_sync(0xffffffffu, incl, 31);
+          if (lane == 0) misc[8] = 1;
         }
-        if (lane == 0) misc[8] = 1;
+        __syncthreads();
       }
-      __syncthreads();
     }
   }
   tc_fence_after();

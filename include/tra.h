@@ -309,6 +309,12 @@ tra_status tra_build_block_mask_ex(const float* r, const float* phi, int heads, 
  *   lse       [heads, N] fp32 natural-log sum of exponentials, or NULL.
  *   row_ptr, col_idx  CSR as written by tra_build_block_mask for the same
  *             heads, N, block_q, block_k (col_idx ascending, no repeats).
+ *             A row whose start is negative or that holds more than nKB
+ *             entries is skipped (O = 0, lse = -inf) and reported through
+ *             tra_get_device_error (TRA_ERR_BAD_INPUT).  With 64-row query
+ *             blocks, where two rows share a tile, a row that is not strictly
+ *             ascending within [0, nKB) is skipped and reported the same way;
+ *             otherwise an entry outside [0, nKB) adds no keys.
  *   d in {64, 128}; block_q, block_k in {16, 64, 128};  when block_q < 128
  *   and either block is 16 tokens, ceil(N / block_k) <= 1024.  scale > 0 and
  *   finite.

@@ -128,3 +128,42 @@ def _c_code():
     code = ctypes.c_int(0)
     s = tra.lib().tra_get_device_error(ctypes.byref(code), tra._stream(None))
     return code.value, s
+
+
+def test_malformed_rows_of_a_two_block_tile_are_skipped():
+    """With 64-row query blocks two CSR rows share a tile and its merged key
+    list.  A row that is not strictly ascending within [0, nKB) (unsorted, a
+    repeated entry, an entry out of range) is skipped and reported, and the
+    other row of its tile is still computed exactly: a skipped row A leaves row
+    B on the merged list, a skipped row B leaves row A on the one-row path."""
+    need_gpu()
+    N, d, B = 1024, 64, 64
+    nb = N // B
+    rows = {q: [q] for q in range(nb)}
+    rows.update({2: [5, 3, 7], 3: [2, 3, 4],      # A unsorted, B kept
+                 4: [0, 4, 9], 5: [1, 1, 4],      # B repeats an entry, A kept
+                 6: [3, nb + 83], 7: [9, 8]})     # both malformed
+    bad = {2, 5, 6, 7}
+    rp, ci = [0], []
+    for q in range(nb):
+        ci += rows[q]
+        rp.append(len(ci))
+    mask = np.zeros((1, nb, nb), bool)
+    for q in range(nb):
+        if q not in bad:
+            mask[0, q, rows[q]] = True
+    g = torch.Generator().manual_seed(11)
+    Q, K, V = (torch.randn(1, N, d, generator=g).to(torch.bfloat16) for _ in range(3))
+    O_ = torch.full((1, N, d), 5.0, dtype=torch.bfloat16, device="cuda")
+    L = torch.empty(1, N, device="cuda")
+    assert tra.tra_get_device_error() == 0
+    tra.tra_block_sparse_attn(Q.cuda(), K.cuda(), V.cuda(), O_, torch.tensor(rp, dtype=torch.int32).cuda(),
+                              torch.tensor(ci, dtype=torch.int32).cuda(), B, B, lse=L)
+    assert _c_code() == (10, 8)
+    Or, Lr = O.sparse_attention(to64(Q), to64(K), to64(V), mask, B, B, 1.0 / math.sqrt(d))
+    for q in bad:
+        assert bool((O_[0, q * B:(q + 1) * B] == 0).all())
+        assert bool(torch.isneginf(L[0, q * B:(q + 1) * B]).all())
+    check_attention(O_, Or, "O with malformed rows")
+    good = np.concatenate([np.arange(q * B, (q + 1) * B) for q in range(nb) if q not in bad])
+    assert np.allclose(to64(L)[0, good], Lr[0, good], atol=1e-3, rtol=0)
