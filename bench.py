@@ -379,7 +379,11 @@ def gpu_arm(args, rank, world, local):
              inputs.perturb(K, wl.seed, c, 1, head_offset=rank * wl.heads)) for c in range(1, calls + 1)]
     log(f"inputs generated in {time.time() - t0:.1f}s")
     host = [Q, K, V] + [x for qk in pert for x in qk]
+    # pinned copies replace the pageable ones (about 8.5 GB per rank at the
+    # 14B shape, so a node running one rank per GPU holds one copy, not two)
     host = [x.pin_memory() for x in host]
+    Q, K, V = host[0], host[1], host[2]
+    del pert
     dev = [x.to(device) for x in host]
     Qd, Kd, Vd = dev[0], dev[1], dev[2]
     sparse_in = [(dev[3 + 2 * i], dev[4 + 2 * i], Vd) for i in range(calls)]
