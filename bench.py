@@ -110,6 +110,17 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def sum_over_ranks(value, device=None):
+    """Sum of a per-rank value over all ranks of the default process group
+    (the value itself without one)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def max_over_ranks(value_ms, device=None):
     """Largest value over all ranks of the default process group (each rank
     times its own work with CUDA events; the job is as slow as its slowest
@@ -489,11 +500,7 @@ def gpu_arm(args, rank, world, local):
     ms_step = elapsed_ms / args.steps
     # whole-job work: every rank calibrates its own tau on its own inputs, so
     # the ranks' kept work differs a little; the job's flops are their sum
-    fl_job = fl_step
-    if world > 1:
-        t = torch.tensor([fl_step], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        fl_job = float(t.item())
+    fl_job = sum_over_ranks(fl_step, device) if world > 1 else fl_step
     value = fl_job / (ms_step * 1e-3) / 1e12
     d_ms, s_ms = statistics.mean(dense_ms), statistics.mean(sparse_ms)
     peaks, peak_kind = load_peaks()

@@ -1,5 +1,5 @@
 """Multi-rank host logic of the bench on CPU (gloo, world size 2): the
-max-over-ranks timing reduction, and per-rank input shards (rank k draws the
+max-over-ranks timing reduction, the sum of the ranks' work, and per-rank input shards (rank k draws the
 heads [k*H, (k+1)*H) of one larger seeded problem, so ranks hold different
 inputs of the same shape)."""
 import os
@@ -29,8 +29,9 @@ def _worker(rank, world, port, out):
     import bench
     from entropy_adaptive_radius_b200 import inputs
     t = bench.max_over_ranks(10.0 + 5.0 * rank)
+    w = bench.sum_over_ranks(1.5 + rank)
     Q, K, V = inputs.make_qkv(2, 3, 4, 2, 8, seed=7, dtype="f32", head_offset=rank * 2)
-    out[rank] = (t, Q.clone(), V.clone())
+    out[rank] = (t, Q.clone(), V.clone(), w)
     dist.barrier()
     dist.destroy_process_group()
 
@@ -44,6 +45,7 @@ def test_max_over_ranks_and_input_shards():
     mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True,
                        start_method="spawn")
     assert out[0][0] == out[1][0] == 15.0
+    assert out[0][3] == out[1][3] == 4.0
     from entropy_adaptive_radius_b200 import inputs
     Q, K, V = inputs.make_qkv(2, 3, 4, 4, 8, seed=7, dtype="f32")
     assert torch.equal(out[0][1], Q[:2]) and torch.equal(out[1][1], Q[2:])
@@ -54,3 +56,4 @@ def test_max_over_ranks_and_input_shards():
 def test_max_over_ranks_without_process_group():
     import bench
     assert bench.max_over_ranks(3.5) == 3.5
+    assert bench.sum_over_ranks(3.5) == 3.5
