@@ -16,10 +16,11 @@
 //                     memory): one softmax warpgroup;
 //   entropy_kernel    the entropy-only pass (no PV, no output).
 // In all of them thread i of a softmax warpgroup owns query row i (TMEM lane
-// i): it reads the score tile S_j, keeps the running max m, Z = sum 2^(u-m)
-// and A = sum 2^(u-m) (u-m) (u = s * log2 e), writes P_j (bf16) to shared
-// memory in the MMA's swizzled layout, rescales O when the max grows by more
-// than 2^8, and finally writes O / Z, the entropy H = ln Z - ln 2 * A / Z and
+// i): it reads the score tile S_j and keeps the running max m, Z = sum 2^(u-m)
+// and A = sum 2^(u-m) (u-m) (u = s * log2 e).  The two attention kernels also
+// write P_j (bf16) to shared memory in the MMA's swizzled layout, rescale O
+// when the max grows by more than 2^8, and finally write O / Z; all three
+// write the entropy H = ln Z - ln 2 * A / Z (dense and entropy-only) and
 // LSE = ln 2 * (m + log2 Z).  The tensor cores compute the next score tile
 // while the softmax of the current one runs.
 //
