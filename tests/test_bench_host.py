@@ -6,8 +6,6 @@ import json
 import os
 
 import numpy as np
-import pytest
-import torch
 
 import bench
 from entropy_adaptive_radius_b200 import inputs, workloads

@@ -8,7 +8,7 @@ import torch
 
 from entropy_adaptive_radius_b200 import inputs, tra, workloads
 from oracle import tra_oracle as O
-from tests.gpu_util import need_gpu, to64
+from tests.gpu_util import need_gpu
 
 pytestmark = pytest.mark.gpu
 

@@ -5,7 +5,6 @@ inputs of the same shape)."""
 import os
 import socket
 
-import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp

@@ -2,10 +2,8 @@
 the E4M3 format written out bit by bit, the per-block quantization against
 its error bound, and FP8 attention against the pinned exact attention on
 inputs that E4M3 represents exactly."""
-import math
 
 import numpy as np
-import pytest
 
 from oracle import tra_oracle as O
 

@@ -1,11 +1,9 @@
 """Pins of the oracle's cross-step reuse schedule (CPU): hand-written plans,
 and schedules that reduce to the pinned dense / sparse attention; plus the
 host-side step sequencing of the layer driver against the oracle's plan."""
-import math
 
 import numpy as np
 import pytest
-import torch
 
 from entropy_adaptive_radius_b200.layer import ReusePolicy
 from oracle import tra_oracle as O
