@@ -1,7 +1,7 @@
 """Multi-rank host logic of the bench on CPU (gloo, world size 2): the
-max-over-ranks timing reduction, the sum of the ranks' work, and per-rank input shards (rank k draws the
-heads [k*H, (k+1)*H) of one larger seeded problem, so ranks hold different
-inputs of the same shape)."""
+max-over-ranks timing reduction, the sum of the ranks' work, and per-rank
+input shards (rank k draws the heads [k*H, (k+1)*H) of one larger seeded
+problem, so ranks hold different inputs of the same shape)."""
 import os
 import socket
 
