@@ -30,12 +30,12 @@ int g_cc_ok[kMaxDevices] = {};  // 0 unknown, 1 sm_100, -1 other
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
 tra_status status_of(cudaError_t e) {
   if (e == cudaSuccess) return TRA_OK;
   return TRA_ERR_CUDA;
 }
-
-}  // namespace
 
 tra_status check_device(std::initializer_list<const void*> ptrs) {
   int dev = 0;
@@ -357,6 +357,10 @@ size_t tra_mask_workspace_size(int heads, tra_grid grid, tra_tile tile, int bloc
   if (heads < 0 || !grid_ok(grid) || !tile_ok(tile) || !block_ok(block_q) || !block_ok(block_k))
     return 0;
   return mask_workspace_bytes(heads, layout_of(grid, tile), block_q, block_k);
+}
+
+size_t tra_workspace_size(int heads, tra_grid grid, int block_q, int block_k) {
+  return tra_mask_workspace_size(heads, grid, tra_tile{1, 4, 4}, block_q, block_k);
 }
 
 tra_status tra_build_block_mask_ex(const float* r, const float* phi, int heads, tra_grid grid,

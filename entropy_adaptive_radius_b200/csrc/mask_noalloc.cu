@@ -79,27 +79,27 @@ extern "C" tra_status tra_build_block_mask_noalloc(const float* r, const float* 
   if (heads > 65535 || static_cast<long long>(heads) * nqb * nkb >= INT_MAX)
     return TRA_ERR_UNSUPPORTED;
   const TileLayout L = layout_of(grid, tile);
-  if (heads > 0 && N > 0) {
-    if (r == nullptr || phi == nullptr || row_ptr == nullptr) return TRA_ERR_INVALID_ARGUMENT;
-    if (col_idx == nullptr && col_capacity > 0) return TRA_ERR_INVALID_ARGUMENT;
-    // Problems whose scratch would not fit the built-in array are refused.
-    if (mask_workspace_bytes(heads, L, block_q, block_k) > kMaskStaticScratchBytes)
-      return TRA_ERR_WORKSPACE;
-  } else if (heads > 0 && row_ptr == nullptr) {
-    return TRA_ERR_INVALID_ARGUMENT;
-  }
-  const tra_status dv = check_device({r, phi, row_ptr, col_idx, nnz});
-  if (dv != TRA_OK) return dv;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (heads == 0 || N == 0) {
+    // The empty problem follows tra_build_block_mask_ex exactly: only row_ptr
+    // and nnz are written, so only they are checked.
+    if (heads > 0 && row_ptr == nullptr) return TRA_ERR_INVALID_ARGUMENT;
+    const tra_status dv = check_device({row_ptr, nnz});
+    if (dv != TRA_OK) return dv;
     cudaError_t e = cudaSuccess;
     if (heads > 0) e = cudaMemsetAsync(row_ptr, 0, sizeof(int) * heads, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(nnz, 0, sizeof(int), st);
-    return e == cudaSuccess ? TRA_OK : TRA_ERR_CUDA;
+    return status_of(e);
   }
+  if (r == nullptr || phi == nullptr || row_ptr == nullptr) return TRA_ERR_INVALID_ARGUMENT;
+  if (col_idx == nullptr && col_capacity > 0) return TRA_ERR_INVALID_ARGUMENT;
+  // Problems whose scratch would not fit the built-in array are refused.
+  if (mask_workspace_bytes(heads, L, block_q, block_k) > kMaskStaticScratchBytes)
+    return TRA_ERR_WORKSPACE;
+  const tra_status dv = check_device({r, phi, row_ptr, col_idx, nnz});
+  if (dv != TRA_OK) return dv;
   void* scratch = scratch_address();
   if (scratch == nullptr) return TRA_ERR_CUDA;
-  const cudaError_t e = launch_block_mask(r, phi, heads, L, block_q, block_k, vote_threshold,
-                                          false, row_ptr, col_idx, col_capacity, nnz, scratch, st);
-  return e == cudaSuccess ? TRA_OK : TRA_ERR_CUDA;
+  return status_of(launch_block_mask(r, phi, heads, L, block_q, block_k, vote_threshold, false,
+                                     row_ptr, col_idx, col_capacity, nnz, scratch, st));
 }

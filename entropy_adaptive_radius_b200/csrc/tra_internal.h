@@ -17,6 +17,9 @@ constexpr int kMaxSide = 16384;    // H, W bound: squared distances stay below 2
 // Device error word of the current device (a module-scope __device__ int).
 int* device_error_word();
 
+// Status of a CUDA runtime result: TRA_OK or TRA_ERR_CUDA (defined in api.cu).
+tra_status status_of(cudaError_t e);
+
 // Argument checks shared by the entry points (defined in api.cu).
 bool grid_ok(const tra_grid& g);  // sides >= 0, within kMaxFrames / kMaxSide, N <= 2^24
 bool tile_ok(const tra_tile& t);  // every tile side >= 1

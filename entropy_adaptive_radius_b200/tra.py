@@ -58,6 +58,7 @@ _PROTOS = {
                                       _c_int, _c_int, _vp]),
     "tra_radial_radius": (_c_int, [_vp, _vp, _c_int, Grid, Tile, _c_float, _c_int, _vp]),
     "tra_mask_workspace_size": (_c_size, [_c_int, Grid, Tile, _c_int, _c_int]),
+    "tra_workspace_size": (_c_size, [_c_int, Grid, _c_int, _c_int]),
     "tra_build_block_mask_ex": (_c_int, [_vp, _vp, _c_int, Grid, Tile, _c_int, _c_int, _c_int,
                                          _c_int, _vp, _vp, _c_ll, _vp, _vp, _c_size, _vp]),
     "tra_build_block_mask": (_c_int, [_vp, _vp, _c_int, Grid, Tile, _c_int, _c_int, _c_int, _vp,
@@ -281,6 +282,11 @@ def _mask_args(heads, grid, block_q, block_k, r, phi, row_ptr, col_idx, nnz, wor
 
 def tra_mask_workspace_size(heads, grid, block_q, block_k, tile=(1, 4, 4)) -> int:
     return int(lib().tra_mask_workspace_size(heads, _grid(grid), _tile(tile), block_q, block_k))
+
+
+def tra_workspace_size(heads, grid, block_q, block_k) -> int:
+    """tra_mask_workspace_size for the default 1 x 4 x 4 tile."""
+    return int(lib().tra_workspace_size(heads, _grid(grid), block_q, block_k))
 
 
 def tra_build_block_mask(r, phi, grid, block_q, block_k, vote, row_ptr, col_idx, nnz, workspace,

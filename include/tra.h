@@ -34,6 +34,12 @@
  *    is skipped (its queries get O = 0, lse = -inf) and recorded the same
  *    way.  No kernel traps.
  *  - Requires a compute capability 10.0 GPU (B200, sm_100a).
+ *  - The library looks up the device addresses of its two module-scope
+ *    objects (the device error word and the scratch array of
+ *    tra_build_block_mask_noalloc) once per device and keeps them.  A
+ *    cudaDeviceReset, or anything else that destroys the device's primary
+ *    context, while the library is loaded leaves those addresses stale: do
+ *    not reset a device between calls into this library.
  */
 #ifndef TRA_H_
 #define TRA_H_
@@ -157,9 +163,17 @@ tra_status tra_budget_radius(const float* H, float* r, float* phi_out, int heads
 
 /*
  * Bytes of device scratch space tra_build_block_mask needs for these sizes
- * (0 if the sizes are invalid).  The space must be 256-byte aligned.
+ * (0 if the sizes are invalid).  The space must be 256-byte aligned.  The
+ * tile is validated like the mask call's; the size itself depends only on
+ * heads, N and the block sizes.
  */
 size_t tra_mask_workspace_size(int heads, tra_grid grid, tra_tile tile, int block_q, int block_k);
+
+/*
+ * The same size without a tile argument: tra_mask_workspace_size with the
+ * 1 frame x 4 rows x 4 columns tile, which gives the size for every tile.
+ */
+size_t tra_workspace_size(int heads, tra_grid grid, int block_q, int block_k);
 
 /*
  * Fused radius mask -> block-sparse CSR (§2 "TRA pipeline", efficient

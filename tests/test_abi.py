@@ -128,6 +128,27 @@ def test_workspace_size_grows_with_problem(L):
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_workspace_size_default_tile(L):
+    """tra_workspace_size is tra_mask_workspace_size with the 1 x 4 x 4 tile,
+    and the size does not depend on the tile."""
+    for heads, grid, bq, bk in ((40, G, 128, 128), (12, tra.Grid(21, 30, 52), 64, 64),
+                                (2, tra.Grid(4, 8, 8), 16, 16), (3, G, 96, 128)):
+        assert L.tra_workspace_size(heads, grid, bq, bk) == L.tra_mask_workspace_size(
+            heads, grid, T, bq, bk)
+    for tile in (tra.Tile(1, 2, 8), tra.Tile(2, 3, 5), tra.Tile(1, 1, 1)):
+        assert L.tra_workspace_size(40, G, 128, 128) == L.tra_mask_workspace_size(
+            40, G, tile, 128, 128)
+
+
+def test_static_scratch_size_matches_the_header():
+    """The binding's copy of TRA_MASK_STATIC_SCRATCH_BYTES is the header's."""
+    m = re.search(r"#define\s+TRA_MASK_STATIC_SCRATCH_BYTES\s+\(([^)]*)\)", open(HEADER).read())
+    assert m, "macro not found"
+    expr = re.sub(r"(\d+)u\b", r"\1", m.group(1))
+    assert re.fullmatch(r"[\d\s*+()]+", expr)
+    assert eval(expr) == tra.MASK_STATIC_SCRATCH_BYTES
+
+
 def test_valid_call_without_gpu_reports_device_error(L):
     # No silent CPU fallback: a well-formed call on a machine without an
     # sm_100 GPU returns TRA_ERR_DEVICE and the binding raises.
@@ -206,4 +227,5 @@ def test_header_compiles_as_c99_and_host_calls_answer(L, tmp_path):
     assert statuses == [tra.status_string(s) for s in range(9)] and len(set(statuses)) == 9
     assert int(kv["workspace"]) == tra.tra_mask_workspace_size(40, (21, 45, 80), 128, 128) > 0
     assert int(kv["workspace_bad"]) == 0
+    assert int(kv["workspace_default_tile"]) == int(kv["workspace"])
     assert int(kv["permute_null"]) == INVALID
