@@ -70,12 +70,14 @@ def margin(Hs, tau, c):
     return worst
 
 
-@pytest.mark.parametrize("refresh,dtype", [("entropy", "bf16"), ("dense", "bf16"), ("entropy", "f32")])
-def test_reuse_loop_matches_oracle_schedule(refresh, dtype):
-    """dtype f32 hands the layer the same (bf16-valued) inputs as float32
-    tensors: its permute then rounds them to bf16, exactly."""
-    need_gpu()
-    steps = make_steps(seed=5)
+def run_schedule(refresh, dtype, layout, seed=5):
+    """The layer's schedule against the oracle's: outputs within the
+    attention tolerances, refreshed entropies within 1e-3, and every rebuilt
+    CSR bit for bit.  With layout "tile_major" the layer is handed the
+    inputs already in tile-major order (permuted on the GPU once, as a model
+    that keeps a transformer block's tokens in that order would) and its
+    outputs are compared in that order."""
+    steps = make_steps(seed=seed)
     policy = ReusePolicy(warmup=1, refresh_every=2, refresh=refresh)
     plan = O.reuse_plan(len(steps), 1, 2, refresh)
     assert [policy.kind(k) for k in range(len(steps))] == plan
@@ -97,14 +99,19 @@ def test_reuse_loop_matches_oracle_schedule(refresh, dtype):
     outs, used, refreshed = O.reuse_run(steps_tm, c, F, tau, gamma32, BQ, BK, 1, plan, scale)
 
     layer = TraLayer((F, HH, WW), HEADS, D, tau=tau, gamma=GAMMA, tile=TILE, block_q=BQ,
-                     block_k=BK, policy=policy)
-    nqb = -(-N // BQ)
+                     block_k=BK, policy=policy, layout=layout)
     for k, (Q, K, V) in enumerate(steps):
         if dtype == "f32":
             Q, K, V = Q.float(), K.float(), V.float()
-        Og = layer(Q.cuda(), K.cuda(), V.cuda())
+        Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+        if layout == "tile_major":
+            Og = layer(layer.to_tile_major(Qd), layer.to_tile_major(Kd), layer.to_tile_major(Vd))
+            ref = outs[k]
+        else:
+            Og = layer(Qd, Kd, Vd)
+            ref = O.inverse_permute(outs[k], pi)
         assert tra.tra_get_device_error() == 0
-        check_attention(Og, O.inverse_permute(outs[k], pi), f"step {k} ({plan[k]})")
+        check_attention(Og, ref, f"step {k} ({plan[k]}, {layout})")
         if plan[k] != "sparse":
             check_close(layer.H, refreshed[k], H_ABS, f"H step {k}")
             mask = O.mask_from_entropy(refreshed[k], c, tau, gamma32, F, BQ, BK, 1)
@@ -118,6 +125,22 @@ def test_reuse_loop_matches_oracle_schedule(refresh, dtype):
     ms = [O.mask_from_entropy(refreshed[k], c, tau, gamma32, F, BQ, BK, 1) for k in refresh_steps]
     assert any(not np.array_equal(ms[0], m) for m in ms[1:])
     assert all(0.0 < m.mean() < 1.0 for m in ms)
+
+
+@pytest.mark.parametrize("refresh,dtype", [("entropy", "bf16"), ("dense", "bf16"), ("entropy", "f32")])
+def test_reuse_loop_matches_oracle_schedule(refresh, dtype):
+    """dtype f32 hands the layer the same (bf16-valued) inputs as float32
+    tensors: its permute then rounds them to bf16, exactly."""
+    need_gpu()
+    run_schedule(refresh, dtype, "original")
+
+
+@pytest.mark.parametrize("refresh", ["entropy", "dense"])
+def test_tile_major_resident_layer_matches_oracle_schedule(refresh):
+    """The resident-layout layer (tokens kept in tile-major order between
+    calls, no per-call permutes) against the oracle's schedule directly."""
+    need_gpu()
+    run_schedule(refresh, "bf16", "tile_major")
 
 
 def test_tile_major_resident_layer_matches_original_layout():
