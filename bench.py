@@ -135,15 +135,14 @@ def max_over_ranks(value_ms, device=None):
     return float(t.item())
 
 
-def workload_config(wl, world, tau=None, kept=None):
-    """The `config` object of the JSON line, the same for both arms: the
-    workload and its shape; tau and the kept fraction as measured (the GPU
-    arm calibrates tau to the workload's target) or the target itself."""
+def workload_config(wl, world):
+    """The `config` object of the JSON line, identical in both arms: the
+    workload's definition (shape, blocks, tile, gamma, vote threshold and the
+    kept-block target tau is calibrated to).  Measured results (tau, kept
+    fraction) are top-level keys of the line."""
     return {"workload": wl.name, "grid": [wl.F, wl.H, wl.W], "N": wl.N, "heads": wl.heads,
             "head_dim": wl.d, "block": [wl.block_q, wl.block_k], "tile": list(wl.tile),
-            "gamma": wl.gamma, "vote": wl.vote,
-            "tau": None if tau is None else round(tau, 6),
-            "kept_fraction": None if kept is None else round(kept, 4),
+            "gamma": wl.gamma, "vote": wl.vote, "kept_target": wl.kept_target,
             "sparse_calls_per_warmup": wl.sparse_calls, "l2": l2_note(wl),
             "parallelism": f"independent x{world}"}
 
@@ -161,11 +160,16 @@ def l2_note(wl):
     return f"inputs fit in L2 ({mb:.1f} MB per tensor); L2 not flushed"
 
 
-def time_ms(fn, reps=5):
+def time_ms(fn, reps=5, flush=None):
+    """Median CUDA-event time of `fn` over `reps` launches after one untimed
+    launch; `flush` (if given) runs before each timed launch, outside the
+    events (an L2 flush)."""
     fn()
     torch.cuda.synchronize()
     ts = []
     for _ in range(reps):
+        if flush is not None:
+            flush()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
         fn()
@@ -387,7 +391,8 @@ def gpu_arm(args, rank, world, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Fourier-feature Q/K of grid position + noise, v ~ N(0,1))",
-        "config": workload_config(wl, world, tau=pipe.tau, kept=kept),
+        "config": workload_config(wl, world),
+        "tau": round(pipe.tau, 8), "kept_fraction": round(kept, 4),
         "sparse_ms_per_call": round(s_ms, 3), "sparse_tflops_kept": round(sparse_tf, 2),
         "dense_ms_per_call": round(d_ms, 3), "dense_tflops": round(dense_tf, 2),
         "mask_ms": round(statistics.mean(mask_ms), 3), "radius_ms": round(statistics.mean(radius_ms), 4),
@@ -415,11 +420,156 @@ def gpu_arm(args, rank, world, local):
                   "ms_per_step": round(e2e["ms"], 3)}
     if rank == 0 and world == 1:
         out["cpu_baseline"] = cpu_baseline(args, Q, K, V, pipe, kept_pairs, fl_step, wl)
+    if world == 1 and wl is workloads.WAN14B and not args.no_configs:
+        del pipe, dev, sparse_in, Qd, Kd, Vd, e2e
+        torch.cuda.empty_cache()
+        out["configs"] = other_configs(device, log)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def l2_flusher(device):
+    """Writes a 256 MB buffer (twice the 126 MB L2) so the next launch starts
+    with a cold L2."""
+    buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    return lambda: buf.fill_(1)
+
+
+def executed_over_kept(row_ptr, col_idx, heads, N, bq, bk):
+    """Work the attention kernel executes over the kept work: with 64-token
+    query blocks a 128-row tile runs the ascending union of its two blocks'
+    key-block lists for all of its rows; otherwise 1."""
+    if bq >= 128:
+        return 1.0
+    nqb = -(-N // bq)
+    rp = row_ptr.reshape(heads, nqb + 1)
+    ksz = np.minimum(bk, N - np.arange(-(-N // bk)) * bk).astype(np.int64)
+    qsz = np.minimum(bq, N - np.arange(nqb) * bq).astype(np.int64)
+    executed = kept = 0
+    for h in range(heads):
+        for t in range(0, nqb, 128 // bq):
+            blocks = range(t, min(nqb, t + 128 // bq))
+            cols = [col_idx[rp[h, b]:rp[h, b + 1]] for b in blocks]
+            union = np.unique(np.concatenate(cols)) if cols else np.zeros(0, np.int64)
+            executed += int(sum(qsz[b] for b in blocks)) * int(ksz[union].sum())
+            kept += sum(int(qsz[b]) * int(ksz[c].sum()) for b, c in zip(blocks, cols))
+    return executed / max(1, kept)
+
+
+def config_point(wl, device, log, peak, flush):
+    """One workload timed in the bench's run: dense warm-up (dense + entropy)
+    call, tau calibrated to the kept target, then the block-sparse call over
+    that CSR, the radius + mask, and (for one sparse call per warm-up) the
+    unamortised entropy + mask overhead.  Kernels are timed alone with CUDA
+    events, L2 flushed before each launch."""
+    from entropy_adaptive_radius_b200 import tra
+    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed, wl.q_scale, wl.dtype)
+    Qd, Kd, Vd = Q.to(device), K.to(device), V.to(device)
+    pipe = Pipeline(wl, device)
+    pipe.warmup_call(Qd, Kd, Vd, None)
+    pipe.tau = calibrate_tau(pipe, wl.kept_target, log)
+    pipe.warmup_call(Qd, Kd, Vd, None)
+    torch.cuda.synchronize()
+    kept = pipe.kept_fraction()
+    rp = pipe.row_ptr.cpu().numpy()
+    ci = pipe.col_idx[: int(pipe.nnz.item())].cpu().numpy()
+    pairs = kept_pair_tokens(rp, ci, wl.heads, wl.N, wl.block_q, wl.block_k)
+    q, k, v, o = pipe.Qtm, pipe.Ktm, pipe.Vtm, pipe.Otm
+    sparse_ms = time_ms(lambda: tra.tra_block_sparse_attn(q, k, v, o, pipe.row_ptr, pipe.col_idx,
+                                                          wl.block_q, wl.block_k), 5, flush)
+    dense_ms = time_ms(lambda: tra.tra_dense_attn_entropy(q, k, v, o, pipe.H), 3, flush)
+    tau = pipe.tau
+    mask_ms = time_ms(lambda: pipe.mask(tau), 5, flush)
+    if tra.tra_get_device_error() != 0:
+        raise RuntimeError("device-side wait timed out")
+    sparse_tf = 4.0 * wl.d * pairs / (sparse_ms * 1e-3) / 1e12
+    dense_tf = 4.0 * wl.d * wl.N * wl.N * wl.heads / (dense_ms * 1e-3) / 1e12
+    cfg = dict(workload_config(wl, 1), l2="L2 flushed before each timed launch")
+    row = {"workload": wl.name, "config": cfg, "tau": round(tau, 8),
+           "kept_fraction": round(kept, 4), "sparse_ms": round(sparse_ms, 3),
+           "sparse_tflops_kept": round(sparse_tf, 1), "sparse_frac": round(sparse_tf / peak, 4),
+           "executed_over_kept": round(executed_over_kept(rp, ci, wl.heads, wl.N, wl.block_q,
+                                                          wl.block_k), 3),
+           "dense_entropy_ms": round(dense_ms, 3), "dense_tflops": round(dense_tf, 1),
+           "dense_frac": round(dense_tf / peak, 4), "mask_plus_radius_ms": round(mask_ms, 3)}
+    if wl.block_q == 128:
+        plain_ms, _, entropy_ms = entropy_overhead_ms(pipe, wl, device, pairs=3)
+        over = max(0.0, entropy_ms) + mask_ms
+        row["entropy_ms"] = round(entropy_ms, 3)
+        row["overhead_ratio_to_sparse_calls"] = round(over / (wl.sparse_calls * sparse_ms), 4)
+    del pipe, Qd, Kd, Vd
+    torch.cuda.empty_cache()
+    return row
+
+
+def sweep_points(device, log, peak, flush, votes, targets):
+    """The density sweep at the 21x45x80, 40-head shape on its own inputs:
+    per vote threshold and target kept fraction, tau calibrated on the
+    warm-up's entropy, then the block-sparse call and the radius + mask
+    timed (L2 flushed before each launch); the 100% point is the dense call."""
+    from entropy_adaptive_radius_b200 import tra
+    wl = workloads.SWEEP
+    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed, wl.q_scale, wl.dtype)
+    Qd, Kd, Vd = Q.to(device), K.to(device), V.to(device)
+    pipe = Pipeline(wl, device)
+    pipe.warmup_call(Qd, Kd, Vd, None)
+    torch.cuda.synchronize()
+    q, k, v, o = pipe.Qtm, pipe.Ktm, pipe.Vtm, pipe.Otm
+    dense_ms = time_ms(lambda: tra.tra_dense_attn_entropy(q, k, v, o, pipe.H), 3, flush)
+    dense_tf = 4.0 * wl.d * wl.N * wl.N * wl.heads / (dense_ms * 1e-3) / 1e12
+    points = []
+    for vote in votes:
+        pipe.vote = vote
+        for target in targets:
+            if target >= 1.0:
+                points.append({"vote": vote, "target_kept": 1.0, "kept_fraction": 1.0,
+                               "path": "dense", "ms": round(dense_ms, 3),
+                               "tflops_kept": round(dense_tf, 1),
+                               "frac": round(dense_tf / peak, 4)})
+                continue
+            tau = calibrate_tau(pipe, target, log)
+            pipe.mask(tau)
+            torch.cuda.synchronize()
+            rp = pipe.row_ptr.cpu().numpy()
+            ci = pipe.col_idx[: int(pipe.nnz.item())].cpu().numpy()
+            pairs = kept_pair_tokens(rp, ci, wl.heads, wl.N, wl.block_q, wl.block_k)
+            ms = time_ms(lambda: tra.tra_block_sparse_attn(q, k, v, o, pipe.row_ptr, pipe.col_idx,
+                                                           wl.block_q, wl.block_k), 3, flush)
+            mask_ms = time_ms(lambda: pipe.mask(tau), 3, flush)
+            tf = 4.0 * wl.d * pairs / (ms * 1e-3) / 1e12
+            points.append({"vote": vote, "target_kept": target,
+                           "kept_fraction": round(pipe.kept_fraction(), 4), "tau": round(tau, 8),
+                           "path": "sparse", "ms": round(ms, 3), "tflops_kept": round(tf, 1),
+                           "frac": round(tf / peak, 4), "speedup_vs_dense": round(dense_ms / ms, 2),
+                           "mask_plus_radius_ms": round(mask_ms, 3)})
+    if tra.tra_get_device_error() != 0:
+        raise RuntimeError("device-side wait timed out")
+    del pipe, Qd, Kd, Vd
+    torch.cuda.empty_cache()
+    return {"workload": wl.name,
+            "config": dict(workload_config(wl, 1), l2="L2 flushed before each timed launch"),
+            "points": points}
+
+
+def other_configs(device, log):
+    """The other workloads, timed in the same run as the headline step: the
+    Wan2.1-1.3B and HunyuanVideo-13B shapes and the density sweep."""
+    peaks, kind = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    flush = l2_flusher(device)
+    t0 = time.time()
+    out = {"peak": f"{peak} TFLOP/s ({kind} bf16 sustained)",
+           "timing": "each kernel alone, CUDA events, median of 3-5 launches, L2 flushed before each"}
+    for key, wl in (("wan13b", workloads.WAN13B), ("hunyuan", workloads.HUNYUAN)):
+        out[key] = config_point(wl, device, log, peak, flush)
+        log(f"config {key} done ({time.time() - t0:.0f}s)")
+    out["sweep"] = sweep_points(device, log, peak, flush, workloads.SWEEP.sweep_votes,
+                                workloads.SWEEP.sweep)
+    log(f"configs done ({time.time() - t0:.0f}s)")
+    return out
 
 
 def e2e_run(pipe, host, dev, calls, args, device, world):
@@ -747,7 +897,9 @@ def reference_arm(args, rank, world):
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(t * 1e3, 1), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": workload_config(wl, world, kept=kept),
+           "config": workload_config(wl, world),
+           "tau": None, "kept_fraction": kept,
+           "note": "the oracle's sampled cost is extrapolated at the workload's kept-block target",
            "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": host_threads(),
                             "kind": "oracle", "sample": sample},
            "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -762,6 +914,8 @@ def kernel_case(args):
     (168 MB per tensor);
     sparse64: the Wan2.1-1.3B shape (12 x 32760 x 128, 64-token blocks) on its
     own radius mask at the calibrated kept fraction;
+    sparse14b: the Wan2.1-14B shape (40 x 75600 x 128, 128-token blocks) on its
+    own radius mask at the calibrated ~12% kept blocks;
     mask: the 21x45x80 grid, 40 heads, radii from entropies near ln N;
     permute: one 21x45x80 x 40-head x 128 bf16 tensor.  Runs the kernel
     `--reps` times and prints the mean CUDA-event time per launch."""
@@ -771,7 +925,29 @@ def kernel_case(args):
     g = torch.Generator(device=dev).manual_seed(0)
     heads, N, d = 40, 16384, 128
     reps = args.reps
-    if args.case == "sparse64":
+    if args.case == "sparse14b":
+        # the Wan2.1-14B shape with its own band mask at the calibrated ~12%
+        # kept blocks; the original-order inputs and output are freed before
+        # the timed launches (about 3.2 GB stays on the device: Q, K, V, O in
+        # tile-major order, the entropy, radii and the CSR)
+        wl = workloads.WAN14B
+        Q, K, V = (t.to(dev) for t in inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed,
+                                                      wl.q_scale, "bf16"))
+        pipe = Pipeline(wl, dev)
+        pipe.warmup_call(Q, K, V, None)
+        pipe.mask(calibrate_tau(pipe, wl.kept_target, lambda m: print(f"[bench] {m}", file=sys.stderr)))
+        torch.cuda.synchronize()
+        del Q, K, V
+        pipe.O = None
+        torch.cuda.empty_cache()
+        rp_h = pipe.row_ptr.cpu().numpy()
+        ci_h = pipe.col_idx.cpu().numpy()
+        flops = 4.0 * wl.d * kept_pair_tokens(rp_h, ci_h, wl.heads, wl.N, wl.block_q, wl.block_k)
+        q, k, v, o = pipe.Qtm, pipe.Ktm, pipe.Vtm, pipe.Otm
+        fn = lambda: tra.tra_block_sparse_attn(q, k, v, o, pipe.row_ptr, pipe.col_idx,  # noqa: E731
+                                               wl.block_q, wl.block_k)
+        unit = ("TFLOP/s", flops / 1e12)
+    elif args.case == "sparse64":
         # the Wan2.1-1.3B shape with its own radius mask (64-token blocks, so
         # each 128-row tile runs the union of two query blocks' rows)
         wl = workloads.WAN13B
@@ -834,7 +1010,8 @@ def kernel_case(args):
         rp = torch.empty(wl.heads * (wl.nqb + 1), dtype=torch.int32, device=dev)
         ci = torch.empty(wl.heads * wl.nqb * wl.nkb, dtype=torch.int32, device=dev)
         nnz = torch.empty(1, dtype=torch.int32, device=dev)
-        fn = lambda: tra.tra_build_block_mask(r, phi, grid, 128, 128, 1, rp, ci, nnz, ws, wl.tile)  # noqa: E731
+        fn = lambda: tra.tra_build_block_mask(r, phi, grid, 128, 128, args.vote, rp, ci, nnz, ws,  # noqa: E731
+                                             wl.tile)
         unit = ("Gpairs/s", wl.heads * wl.N * wl.N / 1e9)
     else:
         wl = WL
@@ -860,10 +1037,11 @@ def kernel_case(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["dense", "sparse", "sparse64", "sparse_fp8", "quant", "entropy", "mask",
+    ap.add_argument("--case", choices=["dense", "sparse", "sparse14b", "sparse64", "sparse_fp8", "quant", "entropy", "mask",
                                        "permute"], default=None,
                     help="run one kernel on a small case (for profiler captures)")
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--vote", type=int, default=1, help="vote threshold of the mask case")
     ap.add_argument("--workload", default="wan14b", choices=sorted(WORKLOADS) + ["sweep", "variants", "reuse"],
                     help="wan14b (default, the headline step), wan13b, hunyuan, tiny, the "
                          "density sweep, the mask variants, or the reuse policies")
@@ -871,6 +1049,9 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="tra", choices=["tra", "reference"])
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads' points (Wan2.1-1.3B, HunyuanVideo, the "
+                         "density sweep) that the 1-GPU line carries under `configs`")
     ap.add_argument("--clocks-csv", default=None,
                     help="where the nvidia-smi clock samples of the timed region go "
                          "({rank} is replaced by the rank); default: a temporary file")

@@ -26,6 +26,22 @@ def test_kept_pair_tokens_counts_tail_blocks_exactly():
     assert expect == sum(km)
 
 
+def test_executed_over_kept_counts_the_union_of_two_query_blocks():
+    """64-token query blocks pair up in 128-row tiles that run the union of
+    their two key-block lists for all 128 rows."""
+    N, B = 256 + 40, 64           # blocks of 64, 64, 64, 64, 40
+    m = np.zeros((1, 5, 5), bool)
+    m[0, 0, 0] = m[0, 1, 1] = True                  # disjoint: union of 2 for 128 rows
+    m[0, 2, [2, 3]] = m[0, 3, [2, 3]] = True        # identical lists: no extra work
+    m[0, 4, [0, 4]] = True                          # last tile holds one 40-row block
+    rp, ci = inputs.csr_from_block_mask(m)
+    kept = 64 * 64 * 2 + 64 * 128 * 2 + 40 * (64 + 40)
+    executed = 128 * 128 + 128 * 128 + 40 * (64 + 40)
+    got = bench.executed_over_kept(rp.ravel(), ci, 1, N, B, B)
+    assert abs(got - executed / kept) < 1e-12
+    assert bench.executed_over_kept(rp.ravel(), ci, 1, N, 128, 128) == 1.0
+
+
 def test_full_csr_keeps_every_block():
     heads, N, B = 3, 1000, 128
     rp, ci = bench.full_csr(heads, N, B, "cpu")
