@@ -26,8 +26,11 @@
 //     counted exactly (lanes over queries): for a query and a key row the
 //     number of keys inside the disk is the overlap of [x_lo, x_hi] with
 //     [x_q - s, x_q + s], s = isqrt(floor(R2) - dy^2); with a vote threshold
-//     of 1 an existence test replaces the count.  Counting stops once the
-//     threshold is reached (only "votes >= threshold" is needed).
+//     of 1 an existence test replaces the count.  Above 1, complete
+//     rectangles are counted in closed form where the disk misses a
+//     rectangle (nothing) or holds all of it (its area), row by row only
+//     where the circle cuts it.  Counting stops once the threshold is reached
+//     (only "votes >= threshold" is needed).
 //  3. scan: exclusive prefix sum of the per-row kept counts -> row_ptr, nnz.
 //  4. compact: kept bits -> ascending col_idx.
 //
@@ -370,6 +373,57 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
             }
           }
           if (__any_sync(0xffffffffu, hit)) word |= 1u << b;
+          continue;
+        }
+        // vote threshold above 1 and complete rectangles: per rectangle, the
+        // queries whose disk holds it whole (its farthest corner inside: the
+        // disk is convex) add its area at once, and the warp stops as soon as
+        // the sum reaches the threshold; only queries whose circle cuts the
+        // rectangle (nearest point inside, farthest corner outside) are then
+        // counted row by row, again stopping at the threshold.
+        if (!exists && nrect >= 0) {
+          const int4* rc = ws.rects + static_cast<size_t>(kb2) * kMaxRect;
+          int votes = 0;
+          for (int i = 0; i < nrect && !keep; ++i) {
+            const int4 rr = rc[i];
+            const int* rs = s_rsq + rr.x * 128 + lane;
+            const int ylo = rr.y >> 16, yhi = rr.y & 0xFFFF;
+            const int xlo = rr.z >> 16, xhi = rr.z & 0xFFFF;
+            const int area = (yhi - ylo + 1) * (xhi - xlo + 1);
+            int cnt = 0, lim[4];
+            uint32_t cut = 0u;  // bit k: query k's circle cuts the rectangle
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              lim[k] = rs[32 * k];
+              const int dxn = max(0, max(xlo - qx[k], qx[k] - xhi));
+              const int dyn = max(0, max(ylo - qy[k], qy[k] - yhi));
+              const int dxf = max(qx[k] - xlo, xhi - qx[k]);
+              const int dyf = max(qy[k] - ylo, yhi - qy[k]);
+              const bool meets = lim[k] >= 0 && dxn * dxn + dyn * dyn <= lim[k];
+              const bool whole = meets && dxf * dxf + dyf * dyf <= lim[k];
+              cnt += whole ? area : 0;
+              cut |= (meets && !whole) ? (1u << k) : 0u;
+            }
+            votes += __reduce_add_sync(0xffffffffu, cnt);
+            keep = votes >= vote;
+            if (keep || !__any_sync(0xffffffffu, cut != 0u)) continue;
+            for (int y = ylo; y <= yhi && !keep; ++y) {
+              int row_cnt = 0;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int dy = y - qy[k];
+                const int m = lim[k] - dy * dy;
+                if (((cut >> k) & 1u) && m >= 0) {
+                  const int sq = isqrt_floor(m);
+                  const int lo = max(xlo, qx[k] - sq), hi = min(xhi, qx[k] + sq);
+                  if (hi >= lo) row_cnt += hi - lo + 1;
+                }
+              }
+              votes += __reduce_add_sync(0xffffffffu, row_cnt);
+              keep = votes >= vote;
+            }
+          }
+          if (keep) word |= 1u << b;
           continue;
         }
       }
