@@ -1,4 +1,4 @@
-"""Chained GPU parity at full size: the whole path as the benchmark runs it,
+"""Chained GPU parity: the whole path as the benchmark runs it,
 through the package's Pipeline (Token Radius Attention summary, §2 "TRA
 pipeline": entropy from one dense warm-up call -> budget -> radius -> fused
 radius mask -> block-sparse attention over the kept blocks, reused by the
@@ -21,6 +21,10 @@ HunyuanVideo-13B, and the density sweep's seed at vote thresholds 1, 4 and
     the whole CSR for validity;
   * every sparse call's O and LSE on the sampled rows, against fp64 sparse
     attention of that call's oracle-permuted inputs over those mask rows.
+
+Three mid-size chains (N = 693 .. 1566, ragged tiles and tails, d = 64 and
+128, blocks of 64 and 128 tokens, vote thresholds 1, 4 and 16) are compared
+with the oracle on every element instead of samples.
 
 The chained check can only compare a stage with the oracle given the GPU's
 own upstream result: an entropy within 1e-3 may move a radius across a token
@@ -195,6 +199,63 @@ def test_chain_full_size(wl):
         o, l_ = ch.sparse(ch.Qd, ch.Kd)
         check_sparse(ch, masks, o, l_, ch.Q, ch.K, "sparse call")
     release(ch)
+
+
+@pytest.mark.parametrize("grid,heads,d,block,vote,gamma", [
+    ((5, 13, 22), 2, 64, 64, 1, 0.3),      # N = 1430: 23 64-blocks, ragged tail of 22 tokens
+    ((3, 18, 29), 3, 128, 128, 4, 0.5),    # N = 1566: 13 128-blocks, ragged tail of 30 tokens
+    ((7, 9, 11), 2, 128, 64, 16, 0.2),     # N = 693: odd query-block count, partial tiles
+])
+def test_chain_mid_size_every_element(grid, heads, d, block, vote, gamma):
+    """The whole chain through the Pipeline at sizes the oracle covers in
+    full: every element of the warm-up's O, H and LSE, every radius, the
+    whole CSR bit for bit (given the GPU's fp32 radii) and every element of
+    two sparse calls on perturbed Q/K over the warm-up's CSR."""
+    need_gpu()
+    wl = workloads.Workload(name=f"mid_{grid}", F=grid[0], H=grid[1], W=grid[2], heads=heads,
+                            d=d, dtype="bf16", block_q=block, block_k=block, gamma=gamma,
+                            vote=vote, seed=11, kept_target=0.3, sparse_calls=2)
+    dev = torch.device("cuda", 0)
+    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, heads, d, wl.seed, wl.q_scale, "bf16")
+    pipe = Pipeline(wl, dev)
+    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    pipe.warmup_call(Qd, Kd, Vd, None)
+    pipe.vote = vote
+    pipe.tau = calibrate_tau(pipe, wl.kept_target)
+    out = torch.empty_like(Qd)
+    lse = torch.empty(heads, wl.N, dtype=torch.float32, device=dev)
+    pipe.warmup_call(Qd, Kd, Vd, None, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert tra.tra_get_device_error() == 0
+    pi = O.tile_major_order(*(wl.F, wl.H, wl.W), wl.tile)
+    c = O.token_coords(wl.F, wl.H, wl.W)[pi]
+    scale = 1.0 / math.sqrt(d)
+    tm = lambda X: O.permute(to64(X), pi)  # noqa: E731
+    Or, Hr, Lr = O.dense_attention_entropy(tm(Q), tm(K), tm(V), scale)
+    check_attention(out, O.inverse_permute(Or, pi), "warm-up O")
+    check_close(pipe.H, Hr, H_ABS, "H")
+    check_close(lse, Lr, LSE_ABS, "LSE")
+    tau32, gamma32 = float(np.float32(pipe.tau)), float(np.float32(gamma))
+    rg, phig, Hg = pipe.r.cpu().numpy(), pipe.phi.cpu().numpy(), to64(pipe.H)
+    for h in range(heads):
+        assert np.allclose(rg[h], O.radius(Hg[h], c[:, 2], tau32, gamma32, wl.F, wl.N),
+                           rtol=2e-6, atol=0)
+    masks = np.stack([O.block_mask(rg[h], phig, c, block, block, vote) for h in range(heads)])
+    rp_ref, ci_ref = O.to_csr(masks)
+    nnz = int(pipe.nnz.item())
+    assert nnz == len(ci_ref) and 0 < nnz < masks.size
+    assert np.array_equal(pipe.row_ptr.cpu().numpy(), rp_ref.ravel())
+    assert np.array_equal(pipe.col_idx[:nnz].cpu().numpy(), ci_ref)
+    for call in (1, 2):
+        Qc, Kc = inputs.perturb(Q, wl.seed, call, 0), inputs.perturb(K, wl.seed, call, 1)
+        o = torch.empty_like(Qd)
+        l_ = torch.empty_like(lse)
+        pipe.sparse_call(Qc.to(dev), Kc.to(dev), Vd, None, out=o, lse=l_)
+        torch.cuda.synchronize()
+        assert tra.tra_get_device_error() == 0
+        Osr, Lsr = O.sparse_attention(tm(Qc), tm(Kc), tm(V), masks, block, block, scale)
+        check_attention(o, O.inverse_permute(Osr, pi), f"sparse call {call} O")
+        check_close(l_, Lsr, LSE_ABS, f"sparse call {call} LSE")
 
 
 @pytest.fixture(scope="module")
