@@ -22,7 +22,7 @@ HunyuanVideo-13B, and the density sweep's seed at vote thresholds 1, 4 and
   * every sparse call's O and LSE on the sampled rows, against fp64 sparse
     attention of that call's oracle-permuted inputs over those mask rows.
 
-Three mid-size chains (N = 693 .. 1566, ragged tiles and tails, d = 64 and
+Three mid-size chains (N = 1430 .. 2064, ragged tiles and tails, d = 64 and
 128, blocks of 64 and 128 tokens, vote thresholds 1, 4 and 16) are compared
 with the oracle on every element instead of samples.
 
@@ -201,12 +201,12 @@ def test_chain_full_size(wl):
     release(ch)
 
 
-@pytest.mark.parametrize("grid,heads,d,block,vote,gamma", [
-    ((5, 13, 22), 2, 64, 64, 1, 0.3),      # N = 1430: 23 64-blocks, ragged tail of 22 tokens
-    ((3, 18, 29), 3, 128, 128, 4, 0.5),    # N = 1566: 13 128-blocks, ragged tail of 30 tokens
-    ((7, 9, 11), 2, 128, 64, 16, 0.2),     # N = 693: odd query-block count, partial tiles
+@pytest.mark.parametrize("grid,heads,d,block,vote,gamma,target", [
+    ((5, 13, 22), 2, 64, 64, 1, 0.3, 0.6),     # N = 1430: 23 64-blocks, ragged tail of 22 tokens
+    ((3, 18, 29), 3, 128, 128, 4, 0.5, 0.55),  # N = 1566: 13 128-blocks, ragged tail of 30 tokens
+    ((3, 16, 43), 2, 128, 64, 16, 0.2, 0.35),  # N = 2064: 33 64-blocks (odd), last one 16 tokens
 ])
-def test_chain_mid_size_every_element(grid, heads, d, block, vote, gamma):
+def test_chain_mid_size_every_element(grid, heads, d, block, vote, gamma, target):
     """The whole chain through the Pipeline at sizes the oracle covers in
     full: every element of the warm-up's O, H and LSE, every radius, the
     whole CSR bit for bit (given the GPU's fp32 radii) and every element of
@@ -214,7 +214,7 @@ def test_chain_mid_size_every_element(grid, heads, d, block, vote, gamma):
     need_gpu()
     wl = workloads.Workload(name=f"mid_{grid}", F=grid[0], H=grid[1], W=grid[2], heads=heads,
                             d=d, dtype="bf16", block_q=block, block_k=block, gamma=gamma,
-                            vote=vote, seed=11, kept_target=0.3, sparse_calls=2)
+                            vote=vote, seed=11, kept_target=target, sparse_calls=2)
     dev = torch.device("cuda", 0)
     Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, heads, d, wl.seed, wl.q_scale, "bf16")
     pipe = Pipeline(wl, dev)
