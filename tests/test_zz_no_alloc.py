@@ -89,3 +89,29 @@ def test_noalloc_refuses_problems_beyond_its_buffer():
     assert s == 3   # TRA_ERR_WORKSPACE, nothing launched
     with pytest.raises(tra.TraError):
         tra._check("tra_build_block_mask_noalloc", s)
+
+
+def test_noalloc_empty_problem_follows_the_workspace_entry_point():
+    """N = 0 (a grid with no frames): both entry points write zero row
+    offsets and nnz = 0, and check only those two outputs, so an unused radius
+    pointer that is not device memory is accepted by both."""
+    need_gpu()
+    heads = 3
+    grid = tra.Grid(0, 45, 80)
+    tile = tra.Tile(1, 4, 4)
+    host_r = (ctypes.c_float * 4)()
+    results = []
+    for noalloc in (False, True):
+        row_ptr = torch.full((heads,), 7, dtype=torch.int32, device="cuda")
+        nnz = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+        rp, nz = ctypes.c_void_p(row_ptr.data_ptr()), ctypes.c_void_p(nnz.data_ptr())
+        r = ctypes.cast(host_r, ctypes.c_void_p)
+        if noalloc:
+            s = tra.lib().tra_build_block_mask_noalloc(r, None, heads, grid, tile, 128, 128, 1, rp,
+                                                      None, 0, nz, ctypes.c_void_p(0))
+        else:
+            s = tra.lib().tra_build_block_mask_ex(r, None, heads, grid, tile, 128, 128, 1, 0, rp,
+                                                 None, 0, nz, None, 0, ctypes.c_void_p(0))
+        torch.cuda.synchronize()
+        results.append((s, row_ptr.cpu().tolist(), int(nnz.item())))
+    assert results[0] == results[1] == (0, [0] * heads, 0)
