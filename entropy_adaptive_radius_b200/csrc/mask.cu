@@ -96,8 +96,12 @@ size_t carve(const TileLayout& L, int heads, int bq, int bk, char* base, MaskWs*
   return rows + info + segs + rects + bits + counts;
 }
 
+// floor(sqrt(m)) for 0 <= m <= 2^30: an estimate from the approximate
+// reciprocal square root (within one of the answer for these m), corrected
+// exactly with integer squares.
 __device__ __forceinline__ int isqrt_floor(int m) {
-  int s = static_cast<int>(sqrtf(static_cast<float>(m)));
+  const float f = static_cast<float>(m);
+  int s = m > 0 ? __float2int_rz(f * rsqrtf(f)) : 0;
   while (s * s > m) --s;
   while ((s + 1) * (s + 1) <= m) ++s;
   return s;
