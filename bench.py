@@ -523,10 +523,12 @@ def sweep_points(device, log, peak, flush, votes, targets):
     points = []
     for vote in votes:
         pipe.vote = vote
+        pipe.mask(1e-12)  # r ~ 0: the kept fraction's floor at this vote threshold
+        floor = round(pipe.kept_fraction(), 4)
         for target in targets:
             if target >= 1.0:
                 points.append({"vote": vote, "target_kept": 1.0, "kept_fraction": 1.0,
-                               "path": "dense", "ms": round(dense_ms, 3),
+                               "kept_floor": floor, "path": "dense", "ms": round(dense_ms, 3),
                                "tflops_kept": round(dense_tf, 1),
                                "frac": round(dense_tf / peak, 4)})
                 continue
@@ -541,7 +543,8 @@ def sweep_points(device, log, peak, flush, votes, targets):
             mask_ms = time_ms(lambda: pipe.mask(tau), 3, flush)
             tf = 4.0 * wl.d * pairs / (ms * 1e-3) / 1e12
             points.append({"vote": vote, "target_kept": target,
-                           "kept_fraction": round(pipe.kept_fraction(), 4), "tau": round(tau, 8),
+                           "kept_fraction": round(pipe.kept_fraction(), 4), "kept_floor": floor,
+                           "tau": round(tau, 8),
                            "path": "sparse", "ms": round(ms, 3), "tflops_kept": round(tf, 1),
                            "frac": round(tf / peak, 4), "speedup_vs_dense": round(dense_ms / ms, 2),
                            "mask_plus_radius_ms": round(mask_ms, 3)})
@@ -721,53 +724,22 @@ def cpu_baseline(args, Q, K, V, pipe, kept_pairs, fl_step, wl):
 
 
 def sweep_arm(args):
-    """Density sweep at the 21x45x80, 40-head shape: for each vote threshold
-    and target kept fraction, tau is bisected to the target (or the nearest
-    reachable fraction: every query keeps its own position in every frame, so
-    the fraction has a floor), then the block-sparse call is timed against the
-    dense calls.  One JSON line per point."""
-    from entropy_adaptive_radius_b200 import tra
+    """Density sweep at the 21x45x80, 40-head shape on its own inputs (the
+    points the default line carries under `configs.sweep`): for each vote
+    threshold and target kept fraction, tau is bisected to the target (or the
+    nearest reachable fraction: every query keeps its own position in every
+    frame, so the fraction has a floor), then the block-sparse call and the
+    radius + mask are timed against the dense call.  One JSON line per point."""
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    wl = workloads.SWEEP
     log = lambda m: print(f"[sweep] {m}", file=sys.stderr, flush=True)  # noqa: E731
-    Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed, wl.q_scale, wl.dtype)
-    Qd, Kd, Vd = Q.to(device), K.to(device), V.to(device)
-    pipe = Pipeline(wl, device)
-    pipe.warmup_call(Qd, Kd, Vd, None)
-    torch.cuda.synchronize()
-    plain_ms, dense_ms, _ = entropy_overhead_ms(pipe, wl, device, pairs=3)
     peaks, kind = load_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    for vote in wl.sweep_votes:
-        pipe.vote = vote
-        pipe.mask(1e-12)
-        floor = pipe.kept_fraction()
-        for target in wl.sweep:
-            if target >= 1.0:
-                ms, kept, tau, pairs = plain_ms, 1.0, None, wl.heads * wl.N * wl.N
-            else:
-                tau = calibrate_tau(pipe, target, log)
-                pipe.mask(tau)
-                kept = pipe.kept_fraction()
-                rp = pipe.row_ptr.cpu().numpy()
-                ci = pipe.col_idx[: int(pipe.nnz.item())].cpu().numpy()
-                pairs = kept_pair_tokens(rp, ci, wl.heads, wl.N, wl.block_q, wl.block_k)
-                ms = time_ms(lambda: tra.tra_block_sparse_attn(
-                    pipe.Qtm, pipe.Ktm, pipe.Vtm, pipe.Otm, pipe.row_ptr, pipe.col_idx,
-                    wl.block_q, wl.block_k), 5)
-                mask_ms = time_ms(lambda: pipe.mask(tau), 3)
-            tf = 4.0 * wl.d * pairs / (ms * 1e-3) / 1e12
-            row = {"workload": wl.name, "vote": vote, "target_kept": target,
-                   "kept_fraction": round(kept, 4), "kept_floor": round(floor, 4),
-                   "tau": None if tau is None else round(tau, 8), "sparse_ms": round(ms, 3),
-                   "sparse_tflops_kept": round(tf, 1), "roofline_frac": round(tf / peak, 4),
-                   "peak": f"{peak} TFLOP/s ({kind} bf16 sustained)",
-                   "dense_entropy_ms": round(dense_ms, 3), "plain_dense_ms": round(plain_ms, 3),
-                   "speedup_vs_dense": round(dense_ms / ms, 3)}
-            if target < 1.0:
-                row["mask_ms"] = round(mask_ms, 3)
-            print(json.dumps(row), flush=True)
+    wl = workloads.SWEEP
+    res = sweep_points(device, log, peak, l2_flusher(device), wl.sweep_votes, wl.sweep)
+    for point in res["points"]:
+        print(json.dumps(dict(workload=res["workload"], peak=f"{peak} TFLOP/s ({kind} bf16 sustained)",
+                              **point)), flush=True)
 
 
 def variants_arm(args):
