@@ -215,13 +215,24 @@ def test_chain_mid_size_every_element(grid, heads, d, block, vote, gamma, target
     wl = workloads.Workload(name=f"mid_{grid}", F=grid[0], H=grid[1], W=grid[2], heads=heads,
                             d=d, dtype="bf16", block_q=block, block_k=block, gamma=gamma,
                             vote=vote, seed=11, kept_target=target, sparse_calls=2)
+    nnz, size = chain_every_element(wl)
+    assert 0 < nnz < size
+
+
+def chain_every_element(wl):
+    """Runs the chain for `wl` (tau calibrated to wl.kept_target, or wl.tau)
+    and compares every output with the oracle; returns (nnz, mask size)."""
+    heads, d, block, vote, gamma = wl.heads, wl.d, wl.block_q, wl.vote, wl.gamma
     dev = torch.device("cuda", 0)
     Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, heads, d, wl.seed, wl.q_scale, "bf16")
     pipe = Pipeline(wl, dev)
     Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
-    pipe.warmup_call(Qd, Kd, Vd, None)
     pipe.vote = vote
-    pipe.tau = calibrate_tau(pipe, wl.kept_target)
+    if wl.kept_target is not None:
+        pipe.warmup_call(Qd, Kd, Vd, None)
+        pipe.tau = calibrate_tau(pipe, wl.kept_target)
+    else:
+        pipe.tau = wl.tau
     out = torch.empty_like(Qd)
     lse = torch.empty(heads, wl.N, dtype=torch.float32, device=dev)
     pipe.warmup_call(Qd, Kd, Vd, None, out=out, lse=lse)
@@ -243,10 +254,10 @@ def test_chain_mid_size_every_element(grid, heads, d, block, vote, gamma, target
     masks = np.stack([O.block_mask(rg[h], phig, c, block, block, vote) for h in range(heads)])
     rp_ref, ci_ref = O.to_csr(masks)
     nnz = int(pipe.nnz.item())
-    assert nnz == len(ci_ref) and 0 < nnz < masks.size
+    assert nnz == len(ci_ref)
     assert np.array_equal(pipe.row_ptr.cpu().numpy(), rp_ref.ravel())
     assert np.array_equal(pipe.col_idx[:nnz].cpu().numpy(), ci_ref)
-    for call in (1, 2):
+    for call in range(1, wl.sparse_calls + 1):
         Qc, Kc = inputs.perturb(Q, wl.seed, call, 0), inputs.perturb(K, wl.seed, call, 1)
         o = torch.empty_like(Qd)
         l_ = torch.empty_like(lse)
@@ -256,6 +267,7 @@ def test_chain_mid_size_every_element(grid, heads, d, block, vote, gamma, target
         Osr, Lsr = O.sparse_attention(tm(Qc), tm(Kc), tm(V), masks, block, block, scale)
         check_attention(o, O.inverse_permute(Osr, pi), f"sparse call {call} O")
         check_close(l_, Lsr, LSE_ABS, f"sparse call {call} LSE")
+    return nnz, masks.size
 
 
 @pytest.fixture(scope="module")
