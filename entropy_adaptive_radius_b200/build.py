@@ -1,6 +1,8 @@
 """Builds libtra.so (the C-ABI library of hand-written sm_100a kernels) in
-the package directory.  Usage: python -m entropy_adaptive_radius_b200.build
-[--force] [--verbose-ptxas]."""
+the package directory, and with --check the checked build libtra_check.so
+(TRA_CHECK: kernels test the indices they derive before using them and report
+an index outside its extent through the device error word).  Usage:
+python -m entropy_adaptive_radius_b200.build [--force] [--verbose-ptxas] [--check]."""
 import argparse
 import concurrent.futures
 import os
@@ -14,6 +16,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libtra.so")
+BUILD_CHECK = os.path.join(ROOT, "_build_check")
+LIB_CHECK = os.path.join(HERE, "libtra_check.so")
 SOURCES = ["api.cu", "permute.cu", "radius.cu", "mask.cu", "attention.cu", "mask_noalloc.cu",
            "quant.cu", "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -46,15 +50,18 @@ def _stale(obj: str, src: str) -> bool:
     return any(os.path.getmtime(p) > t for p in [src] + _headers())
 
 
-def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = False,
+          check: bool = False) -> str:
+    """Compiles the library (check=True: the checked build) and returns its path."""
+    build_dir, lib = (BUILD_CHECK, LIB_CHECK) if check else (BUILD, LIB)
+    os.makedirs(build_dir, exist_ok=True)
     cc = nvcc()
-    flags = _flags(verbose_ptxas)
+    flags = _flags(verbose_ptxas) + (["-DTRA_CHECK"] if check else [])
     jobs = []
     objs = []
     for s in SOURCES:
         src = os.path.join(CSRC, s)
-        obj = os.path.join(BUILD, s.replace(".cu", ".o"))
+        obj = os.path.join(build_dir, s.replace(".cu", ".o"))
         objs.append(obj)
         if force or _stale(obj, src):
             jobs.append([cc, "-c", src, "-o", obj] + flags)
@@ -74,17 +81,18 @@ def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = False)
                 sys.stderr.write(out + "\n")
     if failed:
         raise RuntimeError("nvcc failed")
-    if jobs or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        cmd = [cc, "-shared"] + ARCH + ["-o", LIB] + objs + ["-lcudart_static", "-ldl", "-lrt", "-lpthread"]
+    if jobs or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        cmd = [cc, "-shared"] + ARCH + ["-o", lib] + objs + ["-lcudart_static", "-ldl", "-lrt", "-lpthread"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError("link failed:\n" + r.stdout + r.stderr)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--check", action="store_true", help="build libtra_check.so (TRA_CHECK)")
     a = ap.parse_args()
-    print(build(force=a.force, verbose_ptxas=a.verbose_ptxas))
+    print(build(force=a.force, verbose_ptxas=a.verbose_ptxas, check=a.check))

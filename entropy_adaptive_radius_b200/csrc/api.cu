@@ -437,7 +437,7 @@ tra_status tra_get_device_error(int* code, tra_stream_t stream) {
   }
   *code = v;
   if (v == 0) return TRA_OK;
-  return v == kErrBadCsr ? TRA_ERR_BAD_INPUT : TRA_ERR_TIMEOUT;
+  return (v == kErrBadCsr || v == kErrIndex) ? TRA_ERR_BAD_INPUT : TRA_ERR_TIMEOUT;
 }
 
 }  // extern "C"

@@ -40,6 +40,7 @@
 // n = y * W + x, a key is inside when (n_j - n_i)^2 <= R2, and each query
 // keeps, per key frame, the index interval [n_i - s, n_i + s] with
 // s = isqrt(floor(R2)); boxes and rows are compared as index intervals.
+#include "check.cuh"
 #include "tra_internal.h"
 
 namespace tra {
@@ -58,6 +59,7 @@ struct MaskWs {
   int4* rects;      // [nkb * kMaxRect]: as segs, every position of the rectangle a key of the block
   uint32_t* bits;   // [heads * nqb * nkbw]
   int* counts;      // [heads * nqb]
+  int* err;         // device error word (index checks of the checked build)
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -148,6 +150,7 @@ __global__ void footprint_kernel(TileLayout L, int bk, MaskWs ws) {
       if (rows[i].x == key) { f = i; break; }
     }
     if (f < 0) {
+      if (!in_bounds(nrows, bk, ws.err)) break;
       rows[nrows] = make_uint2(key, (static_cast<uint32_t>(c.x) << 16) | static_cast<uint32_t>(c.x));
       ++nrows;
     } else {
@@ -335,6 +338,7 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
         const int4* sg = ws.segs + static_cast<size_t>(kb) * kMaxSeg;
         for (int i = 0; i < info.y && !survive; ++i) {
           const int4 s = sg[i];
+          if (!in_bounds(s.x, F, ws.err)) continue;
           const int ylo = s.y >> 16, yhi = s.y & 0xFFFF, xlo = s.z >> 16, xhi = s.z & 0xFFFF;
           if constexpr (LINE) {
             const int nlo = ylo * L.W + xlo, nhi = yhi * L.W + xhi;
@@ -365,6 +369,7 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
           bool hit = false;
           for (int i = 0; i < nrect; ++i) {
             const int4 rr = rc[i];
+            if (!in_bounds(rr.x, F, ws.err)) continue;
             const int* rs = s_rsq + rr.x * 128 + lane;
             const int ylo = rr.y >> 16, yhi = rr.y & 0xFFFF;
             const int xlo = rr.z >> 16, xhi = rr.z & 0xFFFF;
@@ -390,6 +395,7 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
           int votes = 0;
           for (int i = 0; i < nrect && !keep; ++i) {
             const int4 rr = rc[i];
+            if (!in_bounds(rr.x, F, ws.err)) continue;
             const int* rs = s_rsq + rr.x * 128 + lane;
             const int ylo = rr.y >> 16, yhi = rr.y & 0xFFFF;
             const int xlo = rr.z >> 16, xhi = rr.z & 0xFFFF;
@@ -439,6 +445,7 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
         bool hit = false;
         for (int i = 0; i < nseg; ++i) {
           const int4 sgm = sg[i];
+          if (!in_bounds(sgm.x, F, ws.err)) continue;
           const int* rs = s_rsq + sgm.x * 128 + lane;
           const int ylo = sgm.y >> 16, yhi = sgm.y & 0xFFFF;
           const int xlo = sgm.z >> 16, xhi = sgm.z & 0xFFFF;
@@ -464,6 +471,7 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
         for (int i = 0; i < nrows; ++i) {
           const uint2 rw = rows[i];
           const int t = static_cast<int>(rw.x >> 16);
+          if (!in_bounds(t, F, ws.err)) continue;
           const int y = static_cast<int>(rw.x & 0xFFFFu);
           const int xlo = static_cast<int>(rw.y >> 16);
           const int xhi = static_cast<int>(rw.y & 0xFFFFu);
@@ -524,6 +532,7 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
         const int p1 = min(N, (kb2 + 1) * bk);
         for (int pp = kb2 * bk; pp < p1 && !keep; ++pp) {
           const Coord c = tile_major_coord(L, pp);
+          if (!in_bounds(c.t, F, ws.err)) continue;
           const int* rs = s_rsq + c.t * 128 + lane;
           int cnt = 0;
 #pragma unroll
@@ -641,6 +650,7 @@ cudaError_t launch_block_mask(const float* r, const float* phi, int heads, const
                               cudaStream_t stream) {
   MaskWs ws;
   carve(L, heads, block_q, block_k, static_cast<char*>(workspace), &ws);
+  ws.err = device_error_word();
   const MaskDims md = mask_dims(L, block_q, block_k);
   footprint_kernel<<<(md.nkb + 127) / 128, 128, 0, stream>>>(L, block_k, ws);
   cudaError_t e = cudaGetLastError();

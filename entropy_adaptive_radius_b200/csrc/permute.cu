@@ -6,6 +6,7 @@
 // chunks, so a warp instruction moves 512 contiguous bytes of output.
 #include <cuda_bf16.h>
 
+#include "check.cuh"
 #include "tra_internal.h"
 
 namespace tra {
@@ -79,7 +80,7 @@ constexpr int kUnroll = 4;
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(kWarps * 32) permute_kernel(const Tin* __restrict__ src,
                                                               Tout* __restrict__ dst, int N, int d,
-                                                              TileLayout L, int inverse) {
+                                                              TileLayout L, int inverse, int* err) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p0 = (blockIdx.x * kWarps + warp) * kRowsPerWarp;
   if (p0 >= N) return;
@@ -97,9 +98,9 @@ __global__ void __launch_bounds__(kWarps * 32) permute_kernel(const Tin* __restr
       const int rr = c / cpr;
       const int cc = c - rr * cpr;
       const int other = __shfl_sync(0xffffffffu, mine, rr < 32 ? rr : 0);
-      if (c < total) {
-        const int srow = inverse ? p0 + rr : other;
-        const int drow = inverse ? other : p0 + rr;
+      const int srow = inverse ? p0 + rr : other;
+      const int drow = inverse ? other : p0 + rr;
+      if (c < total && in_bounds(srow, N, err) && in_bounds(drow, N, err)) {
         move_chunk<Tin, Tout>(src + head_off + static_cast<size_t>(srow) * d + cc * 8,
                               dst + head_off + static_cast<size_t>(drow) * d + cc * 8);
       }
@@ -113,7 +114,8 @@ cudaError_t launch_typed(const void* src, void* dst, int heads, int d, const Til
   const int N = L.F * L.H * L.W;
   const dim3 grid((N + kWarps * kRowsPerWarp - 1) / (kWarps * kRowsPerWarp), heads);
   permute_kernel<Tin, Tout><<<grid, kWarps * 32, 0, stream>>>(
-      static_cast<const Tin*>(src), static_cast<Tout*>(dst), N, d, L, inverse ? 1 : 0);
+      static_cast<const Tin*>(src), static_cast<Tout*>(dst), N, d, L, inverse ? 1 : 0,
+      device_error_word());
   return cudaGetLastError();
 }
 

@@ -25,6 +25,7 @@ enum DeviceError : int {
   kErrWaitPVDone = 9,
   kErrBadCsr = 10,
   kErrSelfTest = 11,  // the self-test's wait on a barrier nothing completes
+  kErrIndex = 12,     // checked builds: an index outside what it indexes (access skipped)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

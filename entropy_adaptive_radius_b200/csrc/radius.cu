@@ -18,6 +18,7 @@
 //    in double and rounded once.
 //  - Radial's static window: r_i = r0 for every query, with the band table
 //    phi_R(delta) = 2^(-b/2) (disk) or 2^(-b) (1D), b = floor(log2(delta + 1)).
+#include "check.cuh"
 #include "tra_internal.h"
 
 namespace tra {
@@ -26,7 +27,7 @@ namespace {
 __global__ void budget_radius_kernel(const float* __restrict__ H, float* __restrict__ r,
                                      float* __restrict__ phi_out, int N, long long total,
                                      TileLayout L, float hexp,
-                                     const __grid_constant__ FrameTables tab) {
+                                     const __grid_constant__ FrameTables tab, int* err) {
   if (phi_out != nullptr && blockIdx.x == 0) {
     for (int t = threadIdx.x; t < L.F; t += blockDim.x) phi_out[t] = tab.phi[t];
   }
@@ -35,6 +36,7 @@ __global__ void budget_radius_kernel(const float* __restrict__ H, float* __restr
        i += stride) {
     const int p = static_cast<int>(i % N);
     const int t = tile_major_coord(L, p).t;
+    if (!in_bounds(t, L.F, err)) continue;
     r[i] = tab.coef[t] * expf(hexp * __ldg(H + i));
   }
 }
@@ -46,7 +48,7 @@ constexpr int kSharedThreads = 1024;
 __global__ void __launch_bounds__(kSharedThreads)
 shared_budget_kernel(const float* __restrict__ H, float* __restrict__ r,
                      float* __restrict__ phi_out, int N, TileLayout L, double tau, bool line,
-                     const __grid_constant__ FrameTablesD tab) {
+                     const __grid_constant__ FrameTablesD tab, int* err) {
   __shared__ double s_part[kSharedThreads / 32];
   const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (phi_out != nullptr && h == 0) {
@@ -67,7 +69,9 @@ shared_budget_kernel(const float* __restrict__ H, float* __restrict__ r,
   const double K = tau * (s_part[0] / static_cast<double>(N));
   float* rh = r + static_cast<size_t>(h) * N;
   for (int i = tid; i < N; i += kSharedThreads) {
-    const double c = tab.c[tile_major_coord(L, i).t];
+    const int t = tile_major_coord(L, i).t;
+    if (!in_bounds(t, L.F, err)) continue;
+    const double c = tab.c[t];
     rh[i] = static_cast<float>(line ? K * c : sqrt(K * c));
   }
 }
@@ -104,7 +108,7 @@ cudaError_t launch_budget_radius(const float* H, float* r, float* phi_out, int h
   const long long total = static_cast<long long>(heads) * N;
   const long long blocks = elementwise_blocks(total);
   budget_radius_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
-      H, r, phi_out, N, total, L, line ? 1.0f : 0.5f, tables);
+      H, r, phi_out, N, total, L, line ? 1.0f : 0.5f, tables, device_error_word());
   return cudaGetLastError();
 }
 
@@ -113,7 +117,7 @@ cudaError_t launch_shared_budget_radius(const float* H, float* r, float* phi_out
                                         const FrameTablesD& tables, cudaStream_t stream) {
   const int N = L.F * L.H * L.W;
   shared_budget_kernel<<<heads, kSharedThreads, 0, stream>>>(H, r, phi_out, N, L, tau, line,
-                                                             tables);
+                                                             tables, device_error_word());
   return cudaGetLastError();
 }
 

@@ -15,7 +15,10 @@ from typing import Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtra.so")
+# The library this binding loads: libtra.so beside this file, or the build
+# that TRA_LIBRARY names (the checked build, libtra_check.so, in the tests).
+LIB_PATH = os.environ.get("TRA_LIBRARY") or os.path.join(_HERE, "libtra.so")
+CHECK_LIB_PATH = os.path.join(_HERE, "libtra_check.so")
 
 TRA_BF16, TRA_F32 = 0, 1
 TRA_METRIC_DISK, TRA_METRIC_LINE = 0, 1

@@ -394,6 +394,9 @@ tra_status tra_selftest_wait_timeout(int limit_ms, int* completed, tra_stream_t 
  *    10      an invalid CSR row (negative start, or longer than nKB; the
  *            row is skipped)                              -> TRA_ERR_BAD_INPUT
  *    11      the self-test's wait (tra_selftest_wait_timeout) -> TRA_ERR_TIMEOUT
+ *    12      checked builds only (libtra_check.so, compiled with TRA_CHECK): an
+ *            index a kernel derived from the layout or from data it read fell
+ *            outside what it indexes; the access was skipped -> TRA_ERR_BAD_INPUT
  * Returns TRA_OK when *code == 0, TRA_ERR_CUDA when the stream reported a
  * CUDA error.
  */

@@ -42,6 +42,15 @@ def test_library_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
 
 
+def test_checked_build_exports_every_declared_symbol():
+    """The index-checked build (libtra_check.so) is the same library."""
+    if not os.path.exists(tra.CHECK_LIB_PATH):
+        tra_build.build(quiet=True, check=True)
+    C = ctypes.CDLL(tra.CHECK_LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(C, name), name
+
+
 def test_status_strings(L):
     for s in range(8):
         assert len(tra.status_string(s)) > 0
