@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
             const int ylo = rr.y >> 16, yhi = rr.y & 0xFFFF;
             const int xlo = rr.z >> 16, xhi = rr.z & 0xFFFF;
             const int area = (yhi - ylo + 1) * (xhi - xlo + 1);
-            int cnt = 0, lim[4];
+            int cnt = 0, own = 0, lim[4];
             uint32_t cut = 0u;  // bit k: query k's circle cuts the rectangle
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -413,9 +413,14 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
               const bool whole = meets && dxf * dxf + dyf * dyf <= lim[k];
               cnt += whole ? area : 0;
               cut |= (meets && !whole) ? (1u << k) : 0u;
+              // a cut query standing inside the rectangle has at least its own
+              // position among its votes (distance 0)
+              own += (meets && !whole && (dxn | dyn) == 0) ? 1 : 0;
             }
             votes += __reduce_add_sync(0xffffffffu, cnt);
             keep = votes >= vote;
+            // exact votes so far plus that lower bound: enough to keep the block
+            if (!keep) keep = votes + __reduce_add_sync(0xffffffffu, own) >= vote;
             if (keep || !__any_sync(0xffffffffu, cut != 0u)) continue;
             for (int y = ylo; y <= yhi && !keep; ++y) {
               int row_cnt = 0;
