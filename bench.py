@@ -179,6 +179,15 @@ def time_ms(fn, reps=5, flush=None):
     return statistics.median(ts)
 
 
+def time_ms_for(fn, seconds, flush=None):
+    """time_ms over as many launches as fill about `seconds` of device time
+    (at least 5): a kernel run back to back that long is in the power-capped
+    steady state the measured sustained peak was taken in."""
+    est = time_ms(fn, 1, flush)
+    reps = int(max(5, min(2000, seconds * 1e3 / max(est, 1e-3))))
+    return time_ms(fn, reps, flush)
+
+
 def code_sha256(path):
     """sha256 of a C++/CUDA source with comments and whitespace removed: it
     changes when the code changes, not when only its comments do."""
@@ -463,8 +472,9 @@ def config_point(wl, device, log, peak, flush):
     """One workload timed in the bench's run: dense warm-up (dense + entropy)
     call, tau calibrated to the kept target, then the block-sparse call over
     that CSR, the radius + mask, and (for one sparse call per warm-up) the
-    unamortised entropy + mask overhead.  Kernels are timed alone with CUDA
-    events, L2 flushed before each launch."""
+    unamortised entropy + mask overhead.  The attention kernels are timed back
+    to back for about a second each (CUDA events per launch, median, L2
+    flushed before each launch), the mask over 5 launches."""
     from entropy_adaptive_radius_b200 import tra
     Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed, wl.q_scale, wl.dtype)
     Qd, Kd, Vd = Q.to(device), K.to(device), V.to(device)
@@ -478,9 +488,10 @@ def config_point(wl, device, log, peak, flush):
     ci = pipe.col_idx[: int(pipe.nnz.item())].cpu().numpy()
     pairs = kept_pair_tokens(rp, ci, wl.heads, wl.N, wl.block_q, wl.block_k)
     q, k, v, o = pipe.Qtm, pipe.Ktm, pipe.Vtm, pipe.Otm
-    sparse_ms = time_ms(lambda: tra.tra_block_sparse_attn(q, k, v, o, pipe.row_ptr, pipe.col_idx,
-                                                          wl.block_q, wl.block_k), 5, flush)
-    dense_ms = time_ms(lambda: tra.tra_dense_attn_entropy(q, k, v, o, pipe.H), 3, flush)
+    sparse_ms = time_ms_for(lambda: tra.tra_block_sparse_attn(q, k, v, o, pipe.row_ptr,
+                                                              pipe.col_idx, wl.block_q,
+                                                              wl.block_k), 1.0, flush)
+    dense_ms = time_ms_for(lambda: tra.tra_dense_attn_entropy(q, k, v, o, pipe.H), 1.0, flush)
     tau = pipe.tau
     mask_ms = time_ms(lambda: pipe.mask(tau), 5, flush)
     if tra.tra_get_device_error() != 0:
@@ -508,8 +519,9 @@ def config_point(wl, device, log, peak, flush):
 def sweep_points(device, log, peak, flush, votes, targets):
     """The density sweep at the 21x45x80, 40-head shape on its own inputs:
     per vote threshold and target kept fraction, tau calibrated on the
-    warm-up's entropy, then the block-sparse call and the radius + mask
-    timed (L2 flushed before each launch); the 100% point is the dense call."""
+    warm-up's entropy, then the block-sparse call (back to back for about half
+    a second) and the radius + mask timed, L2 flushed before each launch; the
+    100% point is the dense call."""
     from entropy_adaptive_radius_b200 import tra
     wl = workloads.SWEEP
     Q, K, V = inputs.make_qkv(wl.F, wl.H, wl.W, wl.heads, wl.d, wl.seed, wl.q_scale, wl.dtype)
@@ -518,7 +530,7 @@ def sweep_points(device, log, peak, flush, votes, targets):
     pipe.warmup_call(Qd, Kd, Vd, None)
     torch.cuda.synchronize()
     q, k, v, o = pipe.Qtm, pipe.Ktm, pipe.Vtm, pipe.Otm
-    dense_ms = time_ms(lambda: tra.tra_dense_attn_entropy(q, k, v, o, pipe.H), 3, flush)
+    dense_ms = time_ms_for(lambda: tra.tra_dense_attn_entropy(q, k, v, o, pipe.H), 1.0, flush)
     dense_tf = 4.0 * wl.d * wl.N * wl.N * wl.heads / (dense_ms * 1e-3) / 1e12
     points = []
     for vote in votes:
@@ -538,8 +550,9 @@ def sweep_points(device, log, peak, flush, votes, targets):
             rp = pipe.row_ptr.cpu().numpy()
             ci = pipe.col_idx[: int(pipe.nnz.item())].cpu().numpy()
             pairs = kept_pair_tokens(rp, ci, wl.heads, wl.N, wl.block_q, wl.block_k)
-            ms = time_ms(lambda: tra.tra_block_sparse_attn(q, k, v, o, pipe.row_ptr, pipe.col_idx,
-                                                           wl.block_q, wl.block_k), 3, flush)
+            ms = time_ms_for(lambda: tra.tra_block_sparse_attn(q, k, v, o, pipe.row_ptr,
+                                                               pipe.col_idx, wl.block_q,
+                                                               wl.block_k), 0.5, flush)
             mask_ms = time_ms(lambda: pipe.mask(tau), 3, flush)
             tf = 4.0 * wl.d * pairs / (ms * 1e-3) / 1e12
             points.append({"vote": vote, "target_kept": target,
@@ -565,7 +578,9 @@ def other_configs(device, log):
     flush = l2_flusher(device)
     t0 = time.time()
     out = {"peak": f"{peak} TFLOP/s ({kind} bf16 sustained)",
-           "timing": "each kernel alone, CUDA events, median of 3-5 launches, L2 flushed before each"}
+           "timing": "attention kernels back to back for about 0.5-1 s each (the sustained peak's "
+                     "method), mask over 3-5 launches; CUDA events per launch, median, L2 flushed "
+                     "before each launch"}
     for key, wl in (("wan13b", workloads.WAN13B), ("hunyuan", workloads.HUNYUAN)):
         out[key] = config_point(wl, device, log, peak, flush)
         log(f"config {key} done ({time.time() - t0:.0f}s)")
