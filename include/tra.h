@@ -63,7 +63,8 @@ typedef enum {
   TRA_ERR_DEVICE = 6,           /* no usable sm_100 device */
   TRA_ERR_TIMEOUT = 7,          /* reported by tra_get_device_error: a wait ran out of time */
   TRA_ERR_BAD_INPUT = 8         /* reported by tra_get_device_error: a kernel met an invalid
-                                   CSR row (negative start, or longer than nKB) */
+                                   CSR row (negative start, or longer than nKB), or (checked
+                                   builds only) an index outside what it indexes */
 } tra_status;
 
 typedef enum { TRA_BF16 = 0, TRA_F32 = 1 } tra_dtype;
