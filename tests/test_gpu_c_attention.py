@@ -215,14 +215,16 @@ def test_full_size_dense_and_sparse_sampled(wl):
     assert (Hn <= math.log(N) + H_ABS).all() and (Hn >= -H_ABS).all()
 
 
-def test_union_list_and_walk_fallback_at_the_cap():
-    """64-row query blocks pair up in 128-row tiles whose key-block list is
-    the merged union of two CSR rows: held in shared memory up to 384
-    entries, walked from the two rows beyond.  Tiles are planted at exactly
-    384 and 385 entries, and with interleaved rows (mixed membership bits) on
-    both sides of the cap; every other row keeps its diagonal block."""
+@pytest.mark.parametrize("d", [64, 128])
+def test_union_list_and_walk_fallback_at_the_cap(d):
+    """At d = 64, 64-row query blocks pair up in 128-row tiles whose
+    key-block list is the merged union of two CSR rows: held in shared memory
+    up to 384 entries, walked from the two rows beyond.  Tiles are planted at
+    exactly 384 and 385 entries, and with interleaved rows (mixed membership
+    bits) on both sides of the cap; every other row keeps its diagonal block.
+    The same at both head dimensions."""
     need_gpu()
-    N, d, B = 32768, 128, 64
+    N, B = 32768, 64
     nb = N // B
     mask = np.zeros((1, nb, nb), bool)
     mask[0, np.arange(nb), np.arange(nb)] = True
