@@ -386,10 +386,11 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
         }
         // vote threshold above 1 and complete rectangles: per rectangle, the
         // queries whose disk holds it whole (its farthest corner inside: the
-        // disk is convex) add its area at once, and the warp stops as soon as
-        // the sum reaches the threshold; only queries whose circle cuts the
-        // rectangle (nearest point inside, farthest corner outside) are then
-        // counted row by row, again stopping at the threshold.
+        // disk is convex) add its area at once, and each query whose circle
+        // cuts it (nearest point inside, farthest corner outside) at least
+        // one vote; the warp stops as soon as that lower bound reaches the
+        // threshold.  Otherwise the cut queries are counted row by row,
+        // again stopping at the threshold.
         if (!exists && nrect >= 0) {
           const int4* rc = ws.rects + static_cast<size_t>(kb2) * kMaxRect;
           int votes = 0;
@@ -413,13 +414,13 @@ __global__ void __launch_bounds__(kVoteThreads) votes_kernel(const float* __rest
               const bool whole = meets && dxf * dxf + dyf * dyf <= lim[k];
               cnt += whole ? area : 0;
               cut |= (meets && !whole) ? (1u << k) : 0u;
-              // a cut query standing inside the rectangle has at least its own
-              // position among its votes (distance 0)
-              own += (meets && !whole && (dxn | dyn) == 0) ? 1 : 0;
+              // a cut query has at least one vote in the rectangle: the
+              // rectangle's nearest point to it is one of its keys, inside
+              own += (meets && !whole) ? 1 : 0;
             }
             votes += __reduce_add_sync(0xffffffffu, cnt);
             keep = votes >= vote;
-            // exact votes so far plus that lower bound: enough to keep the block
+            // exact votes so far plus one per cut query: enough to keep the block
             if (!keep) keep = votes + __reduce_add_sync(0xffffffffu, own) >= vote;
             if (keep || !__any_sync(0xffffffffu, cut != 0u)) continue;
             for (int y = ylo; y <= yhi && !keep; ++y) {
